@@ -1,0 +1,22 @@
+"""Shared pytest setup: the `gpu` marker and on-demand builds of the small C libraries."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _c_libs_built():
+    import oracle
+    import workloads
+    oracle.build()
+    workloads.build()
+    yield
