@@ -1,0 +1,100 @@
+"""ctypes binding of libvtattn.so: the C-ABI entry points under the same names.
+
+Argument marshalling only -- every step of the computation runs in the CUDA
+library.  If the library is missing this module raises at import time; there
+is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvtattn.so")
+
+VT_DTYPE_BF16 = 0
+VT_DTYPE_F32 = 1
+
+VT_OK = 0
+VT_ERR_NULL = 1
+VT_ERR_INVALID_ARG = 2
+VT_ERR_UNSUPPORTED = 3
+VT_ERR_BAD_SEQLENS = 4
+VT_ERR_CUDA = 5
+VT_ERR_DEVICE_TIMEOUT = 6
+
+# every symbol include/vt_attn.h declares
+EXPORTED = (
+    "vt_attn_fwd",
+    "vt_attn_validate_seqlens_host",
+    "vt_attn_smem_bytes",
+    "vt_attn_workspace_bytes",
+    "vt_attn_last_device_status",
+    "vt_attn_status_string",
+    "vt_attn_version",
+)
+
+
+class VtAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libvtattn.so not found at {LIB_PATH}; build it with "
+            "`python -m flash_attention_varlen_b200.build` (nvcc, sm_100a). "
+            "There is no CPU fallback.")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    lib.vt_attn_fwd.argtypes = [P, P, P, P, P, I32, I32, I32, I32, F, ctypes.c_int, P]
+    lib.vt_attn_fwd.restype = ctypes.c_int
+    lib.vt_attn_validate_seqlens_host.argtypes = [P, I32, I32]
+    lib.vt_attn_validate_seqlens_host.restype = ctypes.c_int
+    lib.vt_attn_smem_bytes.argtypes = [I32, ctypes.c_int]
+    lib.vt_attn_smem_bytes.restype = ctypes.c_size_t
+    lib.vt_attn_workspace_bytes.argtypes = [I32, I32, ctypes.c_int]
+    lib.vt_attn_workspace_bytes.restype = ctypes.c_size_t
+    lib.vt_attn_last_device_status.argtypes = [P]
+    lib.vt_attn_last_device_status.restype = ctypes.c_int
+    lib.vt_attn_status_string.argtypes = [ctypes.c_int]
+    lib.vt_attn_status_string.restype = ctypes.c_char_p
+    lib.vt_attn_version.argtypes = []
+    lib.vt_attn_version.restype = I32
+    return lib
+
+
+lib = _load()
+
+
+def vt_attn_fwd(q: int, k: int, v: int, out: int, cu_seqlens: int, num_segments: int,
+                total_tokens: int, H: int, D: int, scale: float, dtype: int, stream: int) -> int:
+    """Raw entry point: device pointers as ints; returns the vt_status code."""
+    return lib.vt_attn_fwd(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D,
+                           ctypes.c_float(scale), dtype, stream)
+
+
+def vt_attn_validate_seqlens_host(cu_seqlens_host: int, num_segments: int, total_tokens: int) -> int:
+    return lib.vt_attn_validate_seqlens_host(cu_seqlens_host, num_segments, total_tokens)
+
+
+def vt_attn_smem_bytes(D: int, dtype: int) -> int:
+    return lib.vt_attn_smem_bytes(D, dtype)
+
+
+def vt_attn_workspace_bytes(num_segments: int, total_tokens: int, dtype: int) -> int:
+    return lib.vt_attn_workspace_bytes(num_segments, total_tokens, dtype)
+
+
+def vt_attn_last_device_status(stream: int) -> int:
+    return lib.vt_attn_last_device_status(stream)
+
+
+def status_string(status: int) -> str:
+    return lib.vt_attn_status_string(status).decode()
+
+
+def vt_attn_version() -> int:
+    return lib.vt_attn_version()

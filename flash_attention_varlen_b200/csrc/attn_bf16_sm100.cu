@@ -1,0 +1,435 @@
+// bf16 varlen attention forward for B200 (sm_100a): TMA + tcgen05 + TMEM.
+//
+// Method: softmax(Q_s K_s^T * scale) V_s per packed segment s (issue #1545
+// (vllm.cpp), "The fix": the block-diagonal mask is a set of per-segment row
+// slices), computed flash-style with a running softmax (PR #1579, "Numerics,
+// both halves"): scores are produced one 128-key tile at a time and never
+// leave the SM.
+//
+// One CTA (persistent, one per SM) works through units of 256 query rows of
+// one (segment, head): two 128-row Q tiles that share every K/V tile.
+//
+//   warp 8  (loader)   : TMA loads Q0/Q1 once per unit and K/V tiles into a
+//                        3-stage ring (64-byte swizzled, 32-column chunks).
+//   warp 9  (MMA)      : one thread issues tcgen05.mma:
+//                          S_i = Q_i K_j^T     (SS, M128 N128 K96)  -> TMEM
+//                          O_i += P_i V_j      (TS, M128 N96 K128; P read from TMEM)
+//                        in the order S0 S1 | PV0 S0' | PV1 S1' | ... so that the
+//                        tensor core works on one tile while the other is in softmax.
+//   warps 0-3, 4-7     : softmax warpgroups for Q0 and Q1, one thread per row:
+//                        tcgen05.ld of the S row, row max, p = 2^(s*c - m) with a
+//                        deferred rescale (the running max m only moves when the
+//                        new tile max exceeds it by more than 8 in log2 units, so
+//                        O in TMEM is rarely touched), P packed to bf16 and written
+//                        back over S in TMEM, then the epilogue O / l -> bf16 -> HBM.
+//
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,352), O1 [384,480);
+// P_i overlays the first 64 columns of S_i (two bf16 per 32-bit column).
+//
+// Keys past the end of a segment inside its last tile are masked (p = 0);
+// query rows past the end are computed but not stored.  Every mbarrier wait is
+// bounded and an abort flag lets all roles leave together.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace vt {
+namespace {
+
+constexpr int kBM = 128;          // query rows per Q tile
+constexpr int kBN = 128;          // keys per K/V tile
+constexpr int kD = 96;            // head width
+constexpr int kStages = 3;        // K/V ring depth
+constexpr int kTileBytes = kBM * kD * 2;   // 24576 (also a 128-key K or V tile)
+constexpr int kChunkBytes = 128 * 64;      // 8192: 128 rows x 32 bf16
+constexpr int kThreads = 320;
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: p stays below 2^8 between rescales
+
+static_assert(kBf16BlockRows == 2 * kBM, "a unit is two Q tiles");
+
+struct Smem {
+  uint8_t q[2][kTileBytes];
+  uint8_t k[kStages][kTileBytes];
+  uint8_t v[kStages][kTileBytes];
+  uint64_t q_full[2];
+  uint64_t q_empty;
+  uint64_t k_full[kStages];
+  uint64_t k_empty[kStages];
+  uint64_t v_full[kStages];
+  uint64_t v_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+
+struct Unit {
+  int head, q0, seg_start, seg_end, nkv;
+  bool has_q1;
+};
+
+__device__ __forceinline__ Unit decode_unit(long long u, int E, const WorkEntry* entries,
+                                            const int32_t* cu) {
+  Unit x;
+  const int e = static_cast<int>(u % E);
+  x.head = static_cast<int>(u / E);
+  const WorkEntry we = entries[e];
+  x.seg_start = cu[we.seg];
+  x.seg_end = cu[we.seg + 1];
+  x.q0 = x.seg_start + we.qblock * (2 * kBM);
+  x.has_q1 = x.q0 + kBM < x.seg_end;
+  x.nkv = (x.seg_end - x.seg_start + kBN - 1) / kBN;
+  return x;
+}
+
+// S = Q K^T: both operands K-major (head dim contiguous), 64-byte swizzle,
+// three 32-column chunks of 8 KB; K = 96 as six K16 steps.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t k_s,
+                                         uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < kD / 16; ++kk) {
+    const uint32_t off = (kk >> 1) * kChunkBytes + (kk & 1) * 32;
+    mma_ss(d_tmem, make_smem_desc(q_s + off, 16, 512, kSwizzle64B),
+           make_smem_desc(k_s + off, 16, 512, kSwizzle64B), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O (+)= P V: P (128 x 128 bf16) from TMEM, V MN-major (head dim contiguous):
+// 8-key groups 512 B apart (SBO), 32-column chunks 8 KB apart (LBO); eight K16 steps.
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_s,
+                                         uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk) {
+    mma_ts(d_tmem, p_tmem + kk * 8, make_smem_desc(v_s + kk * 1024, kChunkBytes, 512, kSwizzle64B),
+           idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Every lane waits; the outcome is made warp-uniform because the tcgen05.ld/st
+// that follow are warp-collective.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* dev_status) {
+  const bool ok = mbar_wait_bounded(bar, parity, abort_flag, dev_status);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                         int head, int row0) {
+#pragma unroll
+  for (int c = 0; c < kD / 32; ++c)
+    tma_load_3d(static_cast<uint8_t*>(dst) + c * kChunkBytes, map, bar, c * 32, head, row0);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, const Bf16Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (raw & 1023u)) & 1023u));
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = a.hdr->num_entries;
+  const long long total = static_cast<long long>(E) * a.H;
+  if (static_cast<long long>(blockIdx.x) >= total) return;  // uniform over the CTA
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], kBM);
+      mbar_init(&sm.o_done[i], 1);
+    }
+    mbar_init(&sm.q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  int* dev_status = a.dev_status;
+
+  if (warp == kWarpLoad) {
+    // ------------------------------------------------------------ loader
+    if (lane == 0) {
+      uint32_t kv_it = 0, unit_it = 0, q0_loads = 0, q1_loads = 0, k_issued = 0, v_issued = 0;
+      bool ok = true;
+      for (long long u = blockIdx.x; u < total && ok; u += gridDim.x, ++unit_it) {
+        const Unit x = decode_unit(u, E, a.entries, a.cu_seqlens);
+        if (unit_it > 0 && !mbar_wait_bounded(&sm.q_empty, (unit_it - 1) & 1, abort_flag, dev_status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&sm.q_full[0], kTileBytes);
+        tma_tile(sm.q[0], &tq, &sm.q_full[0], x.head, x.q0);
+        ++q0_loads;
+        if (x.has_q1) {
+          mbar_arrive_expect_tx(&sm.q_full[1], kTileBytes);
+          tma_tile(sm.q[1], &tq, &sm.q_full[1], x.head, x.q0 + kBM);
+          ++q1_loads;
+        }
+        for (int j = 0; j < x.nkv; ++j, ++kv_it) {
+          const uint32_t st = kv_it % kStages, fill = kv_it / kStages;
+          const int row0 = x.seg_start + j * kBN;
+          if (fill > 0 && !mbar_wait_bounded(&sm.k_empty[st], (fill - 1) & 1, abort_flag, dev_status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
+          tma_tile(sm.k[st], &tk, &sm.k_full[st], x.head, row0);
+          ++k_issued;
+          if (fill > 0 && !mbar_wait_bounded(&sm.v_empty[st], (fill - 1) & 1, abort_flag, dev_status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.v_full[st], kTileBytes);
+          tma_tile(sm.v[st], &tv, &sm.v_full[st], x.head, row0);
+          ++v_issued;
+        }
+      }
+      if (!ok) {
+        // Aborted: let the copies already issued land before the CTA exits.
+        if (q0_loads) mbar_wait_drain(&sm.q_full[0], (q0_loads - 1) & 1);
+        if (q1_loads) mbar_wait_drain(&sm.q_full[1], (q1_loads - 1) & 1);
+        for (uint32_t f = (k_issued > kStages ? k_issued - kStages : 0); f < k_issued; ++f)
+          mbar_wait_drain(&sm.k_full[f % kStages], (f / kStages) & 1);
+        for (uint32_t f = (v_issued > kStages ? v_issued - kStages : 0); f < v_issued; ++f)
+          mbar_wait_drain(&sm.v_full[f % kStages], (f / kStages) & 1);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = a.idesc_qk;
+      const uint32_t idesc_pv = make_idesc_bf16(kBM, kD, false, true, false);
+      const uint32_t q_s0 = smem_u32(sm.q[0]), q_s1 = smem_u32(sm.q[1]);
+      uint32_t kv_it = 0, unit_it = 0, q1_it = 0, p_cnt0 = 0, p_cnt1 = 0;
+      for (long long u = blockIdx.x; u < total; u += gridDim.x, ++unit_it) {
+        const Unit x = decode_unit(u, E, a.entries, a.cu_seqlens);
+        if (!mbar_wait_bounded(&sm.q_full[0], unit_it & 1, abort_flag, dev_status)) break;
+        if (x.has_q1 && !mbar_wait_bounded(&sm.q_full[1], q1_it & 1, abort_flag, dev_status)) break;
+        bool ok = true;
+        {
+          const uint32_t st = kv_it % kStages;
+          if (!mbar_wait_bounded(&sm.k_full[st], (kv_it / kStages) & 1, abort_flag, dev_status)) break;
+          tc_fence_after();
+          const uint32_t k_s = smem_u32(sm.k[st]);
+          issue_qk(tmem + kColS0, q_s0, k_s, idesc_qk);
+          mma_commit(&sm.s_full[0]);
+          if (x.has_q1) {
+            issue_qk(tmem + kColS1, q_s1, k_s, idesc_qk);
+            mma_commit(&sm.s_full[1]);
+          }
+          mma_commit(&sm.k_empty[st]);
+          if (x.nkv == 1) mma_commit(&sm.q_empty);
+        }
+        for (int j = 0; j < x.nkv; ++j) {
+          const uint32_t it = kv_it + j, st = it % kStages;
+          const bool more = j + 1 < x.nkv;
+          const uint32_t st1 = (it + 1) % kStages;
+          const uint32_t v_s = smem_u32(sm.v[st]);
+          if (!mbar_wait_bounded(&sm.p_full[0], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
+          ++p_cnt0;
+          if (!mbar_wait_bounded(&sm.v_full[st], (it / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(tmem + kColO0, tmem + kColS0, v_s, idesc_pv, j > 0);
+          mma_commit(&sm.o_done[0]);
+          if (more) {
+            if (!mbar_wait_bounded(&sm.k_full[st1], ((it + 1) / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
+            tc_fence_after();
+            issue_qk(tmem + kColS0, q_s0, smem_u32(sm.k[st1]), idesc_qk);
+            mma_commit(&sm.s_full[0]);
+          }
+          if (x.has_q1) {
+            if (!mbar_wait_bounded(&sm.p_full[1], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
+            ++p_cnt1;
+            tc_fence_after();
+            issue_pv(tmem + kColO1, tmem + kColS1, v_s, idesc_pv, j > 0);
+            mma_commit(&sm.o_done[1]);
+            if (more) {
+              issue_qk(tmem + kColS1, q_s1, smem_u32(sm.k[st1]), idesc_qk);
+              mma_commit(&sm.s_full[1]);
+            }
+          }
+          mma_commit(&sm.v_empty[st]);
+          if (more) {
+            mma_commit(&sm.k_empty[st1]);
+            if (j + 2 == x.nkv) mma_commit(&sm.q_empty);
+          }
+        }
+        if (!ok) break;
+        kv_it += x.nkv;
+        if (x.has_q1) ++q1_it;
+      }
+      // All MMAs issued by this thread complete before TMEM is released.
+      mma_commit(&sm.drain);
+      mbar_wait_drain(&sm.drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;
+    const int r = tid & 127;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (wg ? kColS1 : kColS0);
+    const uint32_t tO = tmem + lane_base + (wg ? kColO1 : kColO0);
+    const float c = a.scale_log2;
+    uint32_t s_cnt = 0, o_base = 0;
+    for (long long u = blockIdx.x; u < total; u += gridDim.x) {
+      const Unit x = decode_unit(u, E, a.entries, a.cu_seqlens);
+      if (wg == 1 && !x.has_q1) continue;
+      const int row_tok = x.q0 + wg * kBM + r;
+      float m = 0.f, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < x.nkv; ++j) {
+        if (!warp_wait(&sm.s_full[wg], s_cnt & 1, abort_flag, dev_status)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t s[kBN];
+        tmem_ld32(tS + 0, s);
+        tmem_ld32(tS + 32, s + 32);
+        tmem_ld32(tS + 64, s + 64);
+        tmem_ld32(tS + 96, s + 96);
+        tmem_ld_wait();
+        reg_fence<kBN>(s);
+        const int nvalid = x.seg_end - (x.seg_start + j * kBN);  // >= 1
+        float mx = -INFINITY;
+        if (nvalid >= kBN) {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            if (i < nvalid) mx = fmaxf(mx, __uint_as_float(s[i]));
+        }
+        const float mt = mx * c;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m = mt;
+        } else if (mt > m + kRescaleThreshold) {
+          alpha = ex2_approx(m - mt);
+          m = mt;
+          rescale = true;
+        }
+        const float neg_m = -m;
+        float sum0 = 0.f, sum1 = 0.f;
+        uint32_t p[kBN / 2];
+        if (nvalid >= kBN) {
+#pragma unroll
+          for (int i = 0; i < kBN / 2; ++i) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * i]), c, neg_m));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * i + 1]), c, neg_m));
+            sum0 += p0;
+            sum1 += p1;
+            p[i] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < kBN / 2; ++i) {
+            const float p0 = (2 * i < nvalid) ? ex2_approx(fmaf(__uint_as_float(s[2 * i]), c, neg_m)) : 0.f;
+            const float p1 = (2 * i + 1 < nvalid) ? ex2_approx(fmaf(__uint_as_float(s[2 * i + 1]), c, neg_m)) : 0.f;
+            sum0 += p0;
+            sum1 += p1;
+            p[i] = pack_bf16x2(p0, p1);
+          }
+        }
+        l = l * alpha + (sum0 + sum1);
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O must hold PV_{j-1} before it is scaled (the commit behind S_j already
+          // implies it; the wait makes it explicit).
+          if (!warp_wait(&sm.o_done[wg], (o_base + j - 1) & 1, abort_flag, dev_status)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t o[kD];
+          tmem_ld32(tO + 0, o);
+          tmem_ld32(tO + 32, o + 32);
+          tmem_ld32(tO + 64, o + 64);
+          tmem_ld_wait();
+          reg_fence<kD>(o);
+#pragma unroll
+          for (int i = 0; i < kD; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 0, o);
+          tmem_st32(tO + 32, o + 32);
+          tmem_st32(tO + 64, o + 64);
+        }
+        tmem_st32(tS + 0, p);
+        tmem_st32(tS + 32, p + 32);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[wg]);
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16 -> HBM (rows inside the segment only)
+      if (!warp_wait(&sm.o_done[wg], (o_base + x.nkv - 1) & 1, abort_flag, dev_status)) break;
+      tc_fence_after();
+      uint32_t o[kD];
+      tmem_ld32(tO + 0, o);
+      tmem_ld32(tO + 32, o + 32);
+      tmem_ld32(tO + 64, o + 64);
+      tmem_ld_wait();
+      reg_fence<kD>(o);
+      if (row_tok < x.seg_end) {
+        const float inv_l = 1.0f / l;
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) +
+                                              (static_cast<size_t>(row_tok) * a.H + x.head) * (kD * 2));
+#pragma unroll
+        for (int i = 0; i < kD / 8; ++i) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+          w.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+          w.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+          w.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
+          dst[i] = w;
+        }
+      }
+      o_base += x.nkv;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t bf16_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const Bf16Args& args, int grid, cudaStream_t stream) {
+  attn_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, args);
+  return cudaGetLastError();
+}
+
+cudaError_t prepare_attn_bf16() {
+  return cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kSmemBytes));
+}
+
+}  // namespace vt

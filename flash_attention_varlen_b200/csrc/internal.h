@@ -1,0 +1,75 @@
+// Internal interfaces between the C-ABI layer (vt_attn.cu) and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace vt {
+
+// Head of the per-stream scratch buffer, written by the scheduling prepass.
+struct alignas(128) WorkHeader {
+  int32_t status;       // kDevStatus* bit flags of the last call on this scratch
+  int32_t num_entries;  // E: number of (segment, q-block) entries that follow
+  int32_t pad[30];
+};
+
+// A work entry: one block of `block_rows` query rows of one segment.  The
+// kernels expand entry e and head h into unit u = h * E + e.
+struct WorkEntry {
+  int32_t seg;
+  int32_t qblock;
+};
+
+// Entries that a call can produce at most: sum_s ceil(L_s / rows) <= T / rows + n.
+inline int64_t max_work_entries(int64_t total_tokens, int64_t num_segments, int block_rows) {
+  return (total_tokens + block_rows - 1) / block_rows + num_segments;
+}
+
+inline size_t scratch_bytes_for(int64_t total_tokens, int64_t num_segments, int block_rows) {
+  return sizeof(WorkHeader) +
+         static_cast<size_t>(max_work_entries(total_tokens, num_segments, block_rows)) *
+             sizeof(WorkEntry);
+}
+
+// Scheduling prepass (one CTA): validates cu_seqlens, orders segments by
+// length (longest first) and writes the entry list.  Sets status to
+// kDevStatusBadSeqlens and num_entries to 0 on a malformed cu_seqlens.
+cudaError_t launch_schedule(const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                            int32_t block_rows, WorkHeader* hdr, WorkEntry* entries,
+                            cudaStream_t stream);
+
+// bf16 forward on tcgen05 tensor cores (sm_100a).
+constexpr int kBf16BlockRows = 256;  // two 128-row Q tiles per unit
+struct Bf16Args {
+  void* out;
+  const int32_t* cu_seqlens;
+  const WorkHeader* hdr;
+  const WorkEntry* entries;
+  int* dev_status;
+  int32_t H;
+  float scale_log2;    // |scale| * log2(e)
+  uint32_t idesc_qk;   // carries the sign of scale (negated A) for scale < 0
+};
+size_t bf16_smem_bytes();
+cudaError_t prepare_attn_bf16();  // opt in to the kernel's dynamic shared memory (per device)
+cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const Bf16Args& args, int grid, cudaStream_t stream);
+
+// f32 forward on FP32 FMA pipes (exactness arm).
+constexpr int kF32BlockRows = 64;
+struct F32Args {
+  const float* q;
+  const float* k;
+  const float* v;
+  float* out;
+  const int32_t* cu_seqlens;
+  const WorkHeader* hdr;
+  const WorkEntry* entries;
+  int32_t H;
+  float scale_log2;  // scale * log2(e), signed
+};
+size_t f32_smem_bytes();
+cudaError_t launch_attn_f32(const F32Args& args, int grid, cudaStream_t stream);
+
+}  // namespace vt

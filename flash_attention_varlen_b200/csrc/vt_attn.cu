@@ -1,0 +1,262 @@
+// C-ABI entry points of libvtattn (declared in include/vt_attn.h).
+//
+// Host side only: argument validation, the per-(device, stream) scratch
+// buffer that holds the work list, TMA descriptors for the bf16 kernel, and
+// the two launches of a call (scheduling prepass, then the attention kernel).
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "vt_attn.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+constexpr int kHeadDim = 96;
+
+struct DeviceInfo {
+  bool init = false;
+  int num_sms = 0;
+  bool bf16_ready = false;
+};
+
+struct Scratch {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+std::map<std::pair<int, uintptr_t>, Scratch> g_scratch;
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// [T, H, 96] bf16 viewed as (d, h, t); a box is 32 columns x 1 head x 128 rows,
+// stored with the 64-byte swizzle the MMA descriptors expect.
+vt_status make_tensor_map(CUtensorMap* map, const void* base, int32_t T, int32_t H) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return VT_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2,
+                                 static_cast<cuuint64_t>(H) * kHeadDim * 2};
+  const cuuint32_t box[3] = {32, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VT_OK : VT_ERR_CUDA;
+}
+
+vt_status device_info(int dev, DeviceInfo** out) {
+  if (dev < 0 || dev >= kMaxDevices) return VT_ERR_CUDA;
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return VT_ERR_CUDA;
+    d.init = true;
+  }
+  *out = &d;
+  return VT_OK;
+}
+
+// Scratch of at least `need` bytes for (dev, stream); grows by reallocation
+// after draining the stream's earlier work that may still read the old buffer.
+vt_status scratch_for(int dev, cudaStream_t stream, size_t need, Scratch** out) {
+  Scratch& s = g_scratch[{dev, reinterpret_cast<uintptr_t>(stream)}];
+  if (s.bytes < need) {
+    size_t nb = need;
+    if (nb < 2 * s.bytes) nb = 2 * s.bytes;
+    if (nb < (64u << 10)) nb = 64u << 10;
+    if (s.ptr) {
+      if (cudaStreamSynchronize(stream) != cudaSuccess) return VT_ERR_CUDA;
+      cudaFree(s.ptr);
+      s.ptr = nullptr;
+      s.bytes = 0;
+    }
+    if (cudaMalloc(&s.ptr, nb) != cudaSuccess) {
+      s.ptr = nullptr;
+      return VT_ERR_CUDA;
+    }
+    if (cudaMemsetAsync(s.ptr, 0, sizeof(vt::WorkHeader), stream) != cudaSuccess) return VT_ERR_CUDA;
+    s.bytes = nb;
+  }
+  *out = &s;
+  return VT_OK;
+}
+
+int block_rows_for(vt_dtype dtype) {
+  return dtype == VT_DTYPE_BF16 ? vt::kBf16BlockRows : vt::kF32BlockRows;
+}
+
+}  // namespace
+
+extern "C" {
+
+vt_status vt_attn_validate_seqlens_host(const int32_t* cu, int32_t num_segments,
+                                        int32_t total_tokens) {
+  if (!cu) return VT_ERR_NULL;
+  if (num_segments < 0 || total_tokens < 0) return VT_ERR_BAD_SEQLENS;
+  if (cu[0] != 0 || cu[num_segments] != total_tokens) return VT_ERR_BAD_SEQLENS;
+  for (int32_t s = 0; s < num_segments; ++s)
+    if (cu[s + 1] < cu[s]) return VT_ERR_BAD_SEQLENS;
+  return VT_OK;
+}
+
+size_t vt_attn_smem_bytes(int32_t D, vt_dtype dtype) {
+  if (D != kHeadDim) return 0;
+  if (dtype == VT_DTYPE_BF16) return vt::bf16_smem_bytes();
+  if (dtype == VT_DTYPE_F32) return vt::f32_smem_bytes();
+  return 0;
+}
+
+size_t vt_attn_workspace_bytes(int32_t num_segments, int32_t total_tokens, vt_dtype dtype) {
+  if (num_segments < 0 || total_tokens < 0) return 0;
+  if (dtype != VT_DTYPE_BF16 && dtype != VT_DTYPE_F32) return 0;
+  return vt::scratch_bytes_for(total_tokens, num_segments, block_rows_for(dtype));
+}
+
+vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                      const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                      int32_t H, int32_t D, float scale, vt_dtype dtype, void* stream_ptr) {
+  if (dtype != VT_DTYPE_BF16 && dtype != VT_DTYPE_F32) return VT_ERR_INVALID_ARG;
+  if (H < 1 || D < 1 || num_segments < 0 || total_tokens < 0) return VT_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return VT_ERR_INVALID_ARG;
+  if (D != kHeadDim) return VT_ERR_UNSUPPORTED;
+  if (num_segments == 0) return total_tokens == 0 ? VT_OK : VT_ERR_BAD_SEQLENS;
+  if (!cu_seqlens) return VT_ERR_NULL;
+  if (total_tokens == 0) return VT_OK;  // every segment is empty: nothing to write
+  if (!q || !k || !v || !out) return VT_ERR_NULL;
+  const uintptr_t align_or = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                             reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+  if (align_or & 15u) return VT_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(H) * D > (1 << 20)) return VT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) return VT_ERR_INVALID_ARG;
+  const size_t elem = dtype == VT_DTYPE_BF16 ? 2 : 4;
+  const size_t bytes = static_cast<size_t>(total_tokens) * H * D * elem;
+  if (ranges_overlap(out, bytes, q, bytes) || ranges_overlap(out, bytes, k, bytes) ||
+      ranges_overlap(out, bytes, v, bytes))
+    return VT_ERR_INVALID_ARG;
+
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VT_ERR_CUDA;
+  DeviceInfo* di = nullptr;
+  vt_status st = device_info(dev, &di);
+  if (st != VT_OK) return st;
+
+  const int block_rows = block_rows_for(dtype);
+  Scratch* sc = nullptr;
+  st = scratch_for(dev, stream, vt::scratch_bytes_for(total_tokens, num_segments, block_rows), &sc);
+  if (st != VT_OK) return st;
+  auto* hdr = static_cast<vt::WorkHeader*>(sc->ptr);
+  auto* entries = reinterpret_cast<vt::WorkEntry*>(hdr + 1);
+
+  if (vt::launch_schedule(cu_seqlens, num_segments, total_tokens, block_rows, hdr, entries,
+                          stream) != cudaSuccess)
+    return VT_ERR_CUDA;
+
+  const long long max_units =
+      static_cast<long long>(vt::max_work_entries(total_tokens, num_segments, block_rows)) * H;
+  if (dtype == VT_DTYPE_BF16) {
+    if (!di->bf16_ready) {
+      if (vt::prepare_attn_bf16() != cudaSuccess) return VT_ERR_CUDA;
+      di->bf16_ready = true;
+    }
+    CUtensorMap tq, tk, tv;
+    if ((st = make_tensor_map(&tq, q, total_tokens, H)) != VT_OK) return st;
+    if ((st = make_tensor_map(&tk, k, total_tokens, H)) != VT_OK) return st;
+    if ((st = make_tensor_map(&tv, v, total_tokens, H)) != VT_OK) return st;
+    vt::Bf16Args a;
+    a.out = out;
+    a.cu_seqlens = cu_seqlens;
+    a.hdr = hdr;
+    a.entries = entries;
+    a.dev_status = &hdr->status;
+    a.H = H;
+    const double log2e = 1.4426950408889634;
+    a.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(scale)) * log2e);
+    a.idesc_qk = vt::make_idesc_bf16(128, 128, false, false, scale < 0.0f);
+    const int grid = static_cast<int>(max_units < di->num_sms ? max_units : di->num_sms);
+    if (vt::launch_attn_bf16(tq, tk, tv, a, grid, stream) != cudaSuccess) return VT_ERR_CUDA;
+  } else {
+    vt::F32Args a;
+    a.q = static_cast<const float*>(q);
+    a.k = static_cast<const float*>(k);
+    a.v = static_cast<const float*>(v);
+    a.out = static_cast<float*>(out);
+    a.cu_seqlens = cu_seqlens;
+    a.hdr = hdr;
+    a.entries = entries;
+    a.H = H;
+    a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    const long long cap = static_cast<long long>(di->num_sms) * 16;
+    const int grid = static_cast<int>(max_units < cap ? max_units : cap);
+    if (vt::launch_attn_f32(a, grid, stream) != cudaSuccess) return VT_ERR_CUDA;
+  }
+  return VT_OK;
+}
+
+vt_status vt_attn_last_device_status(void* stream_ptr) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VT_ERR_CUDA;
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = g_scratch.find({dev, reinterpret_cast<uintptr_t>(stream)});
+    if (it == g_scratch.end() || !it->second.ptr) return VT_OK;
+    ptr = it->second.ptr;
+  }
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return VT_ERR_CUDA;
+  int status = 0;
+  if (cudaMemcpy(&status, ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return VT_ERR_CUDA;
+  if (status & vt::kDevStatusBadSeqlens) return VT_ERR_BAD_SEQLENS;
+  if (status & vt::kDevStatusTimeout) return VT_ERR_DEVICE_TIMEOUT;
+  return VT_OK;
+}
+
+const char* vt_attn_status_string(vt_status s) {
+  switch (s) {
+    case VT_OK: return "VT_OK";
+    case VT_ERR_NULL: return "VT_ERR_NULL: a required pointer is NULL";
+    case VT_ERR_INVALID_ARG: return "VT_ERR_INVALID_ARG: invalid size, dtype, scale, alignment or aliasing";
+    case VT_ERR_UNSUPPORTED: return "VT_ERR_UNSUPPORTED: head dim other than 96 is not implemented";
+    case VT_ERR_BAD_SEQLENS: return "VT_ERR_BAD_SEQLENS: cu_seqlens must start at 0, not decrease and end at total_tokens";
+    case VT_ERR_CUDA: return "VT_ERR_CUDA: a CUDA call failed";
+    case VT_ERR_DEVICE_TIMEOUT: return "VT_ERR_DEVICE_TIMEOUT: a kernel pipeline wait gave up";
+  }
+  return "unknown vt_status";
+}
+
+int32_t vt_attn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,116 @@
+/*
+ * vt_attn -- varlen block-diagonal attention forward for NVIDIA B200 (sm_100a).
+ *
+ * The operation (issue #1545 (vllm.cpp), "Why this one is bad" and "The fix";
+ * PR #1579, "Numerics, both halves"): the non-causal scaled-dot-product
+ * attention of a vision tower whose tokens are packed into independent
+ * segments.  For every segment s = [cu[s], cu[s+1]), head h, query row i in s:
+ *
+ *     O[i,h,:] = sum_{j in s} softmax_j( scale * <Q[i,h,:], K[j,h,:]> ) V[j,h,:]
+ *
+ * i.e. softmax(Q_s K_s^T * scale) V_s per segment; tokens of different
+ * segments never attend to each other (a block-diagonal mask given as row
+ * slices).  In the perception encoder the pages describe, the segments are
+ * the 32x32-patch windows of a window layer or the whole image of a full
+ * layer; H = 16 heads of width D = 96.
+ *
+ * Layout of q, k, v and out: packed, contiguous, row-major [T, H, D]; element
+ * (t, h, d) sits at index (t*H + h)*D + d.  All four have the same dtype.
+ *
+ * Ownership: the caller owns every buffer.  The library keeps, per
+ * (device, stream), one small scratch buffer for its work list: it is
+ * allocated on the first call on that stream and grown (never shrunk) when a
+ * call needs more; make a first call on a stream before capturing it in a
+ * CUDA graph.  Calls are stream-ordered; calls on different streams use
+ * different scratch buffers.
+ *
+ * Errors: every entry point returns a status and never throws or aborts.
+ * Argument errors are detected on the host before anything is launched.
+ * cu_seqlens lives on the device, so its contents are validated on the device
+ * (before any loop uses them); a malformed cu_seqlens makes the call write
+ * nothing and is reported by vt_attn_last_device_status().
+ */
+#ifndef VT_ATTN_H_
+#define VT_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VT_DTYPE_BF16 = 0, /* bfloat16 inputs/outputs, f32 accumulation (tensor cores) */
+  VT_DTYPE_F32 = 1   /* float32 inputs/outputs, f32 arithmetic (FMA pipes) */
+} vt_dtype;
+
+typedef enum {
+  VT_OK = 0,
+  VT_ERR_NULL = 1,           /* a required pointer is NULL */
+  VT_ERR_INVALID_ARG = 2,    /* bad size, dtype, scale, alignment or aliasing */
+  VT_ERR_UNSUPPORTED = 3,    /* a valid request this build does not implement (D != 96) */
+  VT_ERR_BAD_SEQLENS = 4,    /* cu_seqlens not 0 = cu[0] <= ... <= cu[n] = total_tokens */
+  VT_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed */
+  VT_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up waiting on its own pipeline (bug guard) */
+} vt_status;
+
+/*
+ * Attention forward over packed variable-length segments.
+ *
+ *   q, k, v      device pointers, [total_tokens, H, D] of `dtype`, 16-byte aligned.
+ *   out          device pointer, same shape and dtype; must not overlap q, k or v.
+ *   cu_seqlens   device pointer to num_segments+1 int32 offsets:
+ *                cu[0] = 0, non-decreasing, cu[num_segments] = total_tokens.
+ *                Empty segments are allowed and produce no rows.
+ *   num_segments >= 0; total_tokens >= 0 (both 0, or total_tokens 0: no work).
+ *   H            heads, >= 1 (the encoder uses 16).
+ *   D            head width; only 96 is implemented (VT_ERR_UNSUPPORTED otherwise).
+ *   scale        any finite float (the encoder uses 1/sqrt(96)).
+ *   stream       cudaStream_t as an opaque pointer (NULL = legacy default stream).
+ *
+ * Asynchronous: returns once the work is queued on `stream`.
+ */
+vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                      const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                      int32_t H, int32_t D, float scale, vt_dtype dtype, void* stream);
+
+/*
+ * Pure host check of a host copy of cu_seqlens (num_segments+1 entries):
+ * VT_OK, VT_ERR_NULL or VT_ERR_BAD_SEQLENS.  Touches no GPU.
+ */
+vt_status vt_attn_validate_seqlens_host(const int32_t* cu_seqlens_host, int32_t num_segments,
+                                        int32_t total_tokens);
+
+/*
+ * Dynamic shared memory one CTA of the forward kernel for (D, dtype) uses, in
+ * bytes; 0 for an unsupported combination.  Pure host arithmetic: the launch
+ * shape contract, testable without a GPU (PR #1578 keeps the same kind of
+ * host-side shared-memory contract next to its flash kernel).
+ */
+size_t vt_attn_smem_bytes(int32_t D, vt_dtype dtype);
+
+/*
+ * Bytes of scratch a call with these sizes needs (the work list).  Pure host.
+ */
+size_t vt_attn_workspace_bytes(int32_t num_segments, int32_t total_tokens, vt_dtype dtype);
+
+/*
+ * Synchronises `stream` and reports what the device side of the last
+ * vt_attn_fwd call on it found: VT_OK, VT_ERR_BAD_SEQLENS or
+ * VT_ERR_DEVICE_TIMEOUT (VT_ERR_CUDA if the synchronisation itself failed;
+ * VT_OK if no call was made on this stream).
+ */
+vt_status vt_attn_last_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* vt_attn_status_string(vt_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t vt_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VT_ATTN_H_ */

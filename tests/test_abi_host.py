@@ -1,0 +1,119 @@
+"""Host-side checks of the C-ABI library that need no GPU.
+
+The library must load, export every entry point ``include/vt_attn.h``
+declares, and reject bad arguments on the host before touching a device.
+Only calls that fail host validation are made here, so nothing is launched.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def binding():
+    from flash_attention_varlen_b200 import build as b
+    b.build()
+    from flash_attention_varlen_b200 import _binding
+    return _binding
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "vt_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(vt_attn_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(binding):
+    declared = _declared_functions()
+    assert declared, "no declarations parsed"
+    assert sorted(binding.EXPORTED) == declared
+    for name in declared:
+        assert hasattr(binding.lib, name), name
+    # and the names are real dynamic symbols of the .so
+    out = os.popen(f"nm -D --defined-only {binding.LIB_PATH}").read()
+    for name in declared:
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def _cu(arr):
+    a = np.ascontiguousarray(arr, dtype=np.int32)
+    return a, a.ctypes.data
+
+
+def test_validate_seqlens_host(binding):
+    ok = binding.VT_OK
+    bad = binding.VT_ERR_BAD_SEQLENS
+    a, p = _cu([0, 5, 5, 12])
+    assert binding.vt_attn_validate_seqlens_host(p, 3, 12) == ok
+    a, p = _cu([0])
+    assert binding.vt_attn_validate_seqlens_host(p, 0, 0) == ok
+    for arr, n, T in (([1, 5], 1, 5), ([0, 5], 1, 6), ([0, 6, 5, 9], 3, 9), ([0, 3], 1, 3)):
+        a, p = _cu(arr)
+        want = ok if (arr == [0, 3]) else bad
+        assert binding.vt_attn_validate_seqlens_host(p, n, T) == want
+    assert binding.vt_attn_validate_seqlens_host(None, 1, 1) == binding.VT_ERR_NULL
+    a, p = _cu([0, 4])
+    assert binding.vt_attn_validate_seqlens_host(p, -1, 4) == bad
+
+
+def test_smem_contract(binding):
+    b = binding.vt_attn_smem_bytes(96, binding.VT_DTYPE_BF16)
+    f = binding.vt_attn_smem_bytes(96, binding.VT_DTYPE_F32)
+    # bf16: 2 Q tiles + 3-stage K and V rings of 128 x 96 bf16 tiles, plus barriers and
+    # 1 KB alignment slack; must fit the 227 KB per-CTA opt-in limit of sm_100
+    assert 8 * 128 * 96 * 2 < b <= 232448
+    assert f == 2 * 32 * 96 * 4 and f <= 48 * 1024
+    assert binding.vt_attn_smem_bytes(64, binding.VT_DTYPE_BF16) == 0
+    assert binding.vt_attn_smem_bytes(96, 7) == 0
+
+
+def test_workspace_bytes(binding):
+    # header (128 B) + 8 B per entry, entries <= ceil(T / rows) + n
+    assert binding.vt_attn_workspace_bytes(16, 16384, binding.VT_DTYPE_BF16) == 128 + 8 * (64 + 16)
+    assert binding.vt_attn_workspace_bytes(1, 256, binding.VT_DTYPE_F32) == 128 + 8 * (4 + 1)
+    assert binding.vt_attn_workspace_bytes(-1, 5, binding.VT_DTYPE_BF16) == 0
+
+
+def test_status_strings_and_version(binding):
+    for code in range(7):
+        s = binding.status_string(code)
+        assert s.startswith("VT_")
+    assert binding.status_string(99) == "unknown vt_status"
+    assert binding.vt_attn_version() >= 100
+
+
+def test_fwd_rejects_bad_arguments_on_host(binding):
+    f = binding.vt_attn_fwd
+    cu, cup = _cu([0, 4])
+    P = 4096  # fake, 16-byte aligned, never dereferenced: every call below fails host checks
+    BF, F32 = binding.VT_DTYPE_BF16, binding.VT_DTYPE_F32
+    assert f(P, P, P, P * 16, cup, 1, 4, 16, 64, 0.1, BF, 0) == binding.VT_ERR_UNSUPPORTED
+    assert f(P, P, P, P * 16, cup, 1, 4, 16, 96, 0.1, 5, 0) == binding.VT_ERR_INVALID_ARG
+    assert f(P, P, P, P * 16, cup, 1, 4, 0, 96, 0.1, BF, 0) == binding.VT_ERR_INVALID_ARG
+    assert f(P, P, P, P * 16, cup, 1, 4, 16, 96, float("nan"), BF, 0) == binding.VT_ERR_INVALID_ARG
+    assert f(P, P, P, P * 16, cup, 1, 4, 16, 96, float("inf"), F32, 0) == binding.VT_ERR_INVALID_ARG
+    assert f(P, P, P, P * 16, cup, -1, 4, 16, 96, 0.1, BF, 0) == binding.VT_ERR_INVALID_ARG
+    # no segments: fine with no tokens, inconsistent otherwise
+    assert f(0, 0, 0, 0, 0, 0, 0, 16, 96, 0.1, BF, 0) == binding.VT_OK
+    assert f(0, 0, 0, 0, 0, 0, 8, 16, 96, 0.1, BF, 0) == binding.VT_ERR_BAD_SEQLENS
+    # all segments empty: no work, no launch
+    assert f(0, 0, 0, 0, cup, 3, 0, 16, 96, 0.1, BF, 0) == binding.VT_OK
+    assert f(P, P, P, P * 16, 0, 1, 4, 16, 96, 0.1, BF, 0) == binding.VT_ERR_NULL
+    assert f(0, P, P, P * 16, cup, 1, 4, 16, 96, 0.1, BF, 0) == binding.VT_ERR_NULL
+    # misaligned pointers and aliasing of out with an input
+    assert f(P + 2, P, P, P * 16, cup, 1, 4, 16, 96, 0.1, BF, 0) == binding.VT_ERR_INVALID_ARG
+    assert f(P, P * 8, P * 12, P + 64, cup, 1, 4, 16, 96, 0.1, BF, 0) == binding.VT_ERR_INVALID_ARG
+
+
+def test_python_wrapper_refuses_cpu_tensors(binding):
+    import torch
+    from flash_attention_varlen_b200 import attn_fwd
+    q = torch.zeros(4, 16, 96, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        attn_fwd(q, q, q, cu)

@@ -1,0 +1,282 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the f64 CPU oracle.
+
+Tolerances (fixed by the workload definition, applied element by element to
+the GPU output widened to f64):
+  bf16 in/out, f32 accumulation : max-abs <= 1e-2 and mean-abs <= 1e-3
+  f32  in/out                   : max-abs <= 1e-5
+and no NaN/Inf anywhere.  Inputs are the seeded workloads of ``workloads``;
+small cases are compared in full, the large ones (4096-token full layer,
+varlen batch, the 16384-token tower the benchmark times) on sampled
+(token, head) rows the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+BF16_MAX, BF16_MEAN, F32_MAX = 1e-2, 1e-3, 1e-5
+SCALE = 1.0 / math.sqrt(96)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from flash_attention_varlen_b200 import build
+    build.build()
+
+
+def _to_dev(a, dtype):
+    if dtype == "bf16":
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.cuda()
+
+
+def _run(q, k, v, cu, dtype, scale=SCALE, H=None):
+    import flash_attention_varlen_b200 as fa
+    dq, dk, dv = (_to_dev(x, dtype) for x in (q, k, v))
+    dcu = torch.from_numpy(np.ascontiguousarray(cu, dtype=np.int32)).cuda()
+    out = fa.attn_fwd(dq, dk, dv, dcu, scale=scale)
+    fa.check_device_status()
+    return out.float().cpu().numpy().astype(np.float64)
+
+
+def _check(got, ref, dtype, what):
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    if dtype == "bf16":
+        assert err.max() <= BF16_MAX, f"{what}: max-abs {err.max():.3e}"
+        assert err.mean() <= BF16_MEAN, f"{what}: mean-abs {err.mean():.3e}"
+    else:
+        assert err.max() <= F32_MAX, f"{what}: max-abs {err.max():.3e}"
+    return float(err.max()), float(err.mean())
+
+
+def _full_case(case, scale=SCALE):
+    q, k, v = case.inputs()
+    got = _run(q, k, v, case.cu_seqlens, case.dtype, scale)
+    ref = oracle.attn_fwd(q, k, v, case.cu_seqlens, scale)
+    return _check(got, ref, case.dtype, case.name)
+
+
+def _sample_rows(T, H, n, seed):
+    rng = np.random.default_rng(seed)
+    tok = rng.integers(0, T, n)
+    head = rng.integers(0, H, n)
+    # always include both ends of the packed tensor
+    tok[:H] = 0
+    head[:H] = np.arange(H)
+    tok[H:2 * H] = T - 1
+    head[H:2 * H] = np.arange(H)
+    return tok.astype(np.int32), head.astype(np.int32)
+
+
+def _sampled_case(case, n_rows=2048, scale=SCALE, seed=0):
+    q, k, v = case.inputs()
+    got = _run(q, k, v, case.cu_seqlens, case.dtype, scale)
+    tok, head = _sample_rows(case.T, case.H, n_rows, seed)
+    ref = oracle.attn_rows(q, k, v, case.cu_seqlens, scale, tok, head)
+    return _check(got[tok, head], ref, case.dtype, case.name)
+
+
+# ---------------------------------------------------------------- the five workloads
+
+def test_tiny256_bf16():
+    _full_case(workloads.tiny_case("bf16"))
+
+
+def test_tiny256_f32():
+    _full_case(workloads.tiny_case("f32"))
+
+
+@pytest.mark.parametrize("peaked", [False, True])
+def test_image448(peaked):
+    _full_case(workloads.image448_case(peaked))
+
+
+def test_image896_window_layer():
+    _full_case(workloads.image896_cases()[0])
+
+
+def test_image896_full_layer():
+    _sampled_case(workloads.image896_cases()[1], n_rows=4096)
+
+
+def test_varlen8_images():
+    _sampled_case(workloads.varlen8_case(), n_rows=4096)
+
+
+def test_tower16k_every_layer():
+    """All 50 layers of the 16384-token tower, as the benchmark runs them, on sampled rows."""
+    for case in workloads.tower_cases():
+        _sampled_case(case, n_rows=96, seed=case.seed)
+
+
+# ---------------------------------------------------------------- edge cases
+
+RAGGED = [1, 127, 128, 0, 129, 255, 256, 257, 2, 383, 511, 640, 0]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_ragged_segments(dtype):
+    cu = workloads.cu_from_lengths(RAGGED)
+    case = workloads.Case(f"ragged_{dtype}", cu, seed=3, dtype=dtype)
+    _full_case(case)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("H", [1, 3])
+def test_other_head_counts(dtype, H):
+    case = workloads.Case(f"H{H}_{dtype}", workloads.cu_from_lengths([300, 77, 129]), seed=4,
+                          dtype=dtype, H=H)
+    _full_case(case)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("scale", [0.0, -0.25, 0.5])
+def test_scales(dtype, scale):
+    case = workloads.Case(f"scale_{dtype}", workloads.cu_from_lengths([200, 333]), seed=5, dtype=dtype)
+    _full_case(case, scale=scale)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_single_key_segments_return_v_exactly(dtype):
+    cu = workloads.cu_from_lengths([1, 1, 5, 1, 1])
+    case = workloads.Case("single", cu, seed=6, dtype=dtype)
+    q, k, v = case.inputs()
+    got = _run(q, k, v, cu, dtype)
+    vv = workloads.bf16_bits_to_f32(v) if dtype == "bf16" else v
+    for t in (0, 1, 7, 8):
+        assert np.array_equal(got[t], vv[t].astype(np.float64))
+
+
+def test_identical_keys_give_mean_of_values():
+    T = 700
+    case = workloads.Case("idk", workloads.cu_from_lengths([T]), seed=7, dtype="bf16")
+    q, k, v = case.inputs()
+    k[:] = k[0]
+    got = _run(q, k, v, case.cu_seqlens, "bf16")
+    mean = workloads.bf16_bits_to_f32(v).astype(np.float64).mean(axis=0)
+    _check(got, np.broadcast_to(mean, got.shape), "bf16", "identical keys")
+
+
+def test_deferred_rescale_ramp():
+    """Logits grow along the key axis so the running max crosses the rescale threshold often."""
+    T, H, D = 1536, 2, 96
+    q = np.zeros((T, H, D), np.float32)
+    k = np.zeros((T, H, D), np.float32)
+    q[:, :, 0] = 4.0
+    ramp = np.linspace(-6.0, 30.0, T, dtype=np.float32)
+    k[:, :, 0] = ramp[:, None]
+    k[:, :, 1] = (np.arange(T) % 7 - 3).astype(np.float32)[:, None] * 0.5
+    q[:, :, 1] = 1.0
+    rng = np.random.default_rng(8)
+    v = rng.normal(size=(T, H, D)).astype(np.float32)
+    cu = workloads.cu_from_lengths([T // 2, T // 2])
+    for dtype in ("bf16", "f32"):
+        if dtype == "bf16":
+            qq, kk, vv = (_round_bf16(x) for x in (q, k, v))
+        else:
+            qq, kk, vv = q, k, v
+        got = _run(qq, kk, vv, cu, dtype, scale=1.0)
+        ref = oracle.attn_fwd(qq, kk, vv, cu, 1.0)
+        _check(got, ref, dtype, f"ramp_{dtype}")
+
+
+def _round_bf16(x):
+    u = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def test_block_diagonal_independence_and_packing_order_bitwise():
+    lens = [300, 1024, 77, 513]
+    cu = workloads.cu_from_lengths(lens)
+    case = workloads.Case("indep", cu, seed=9, dtype="bf16")
+    q, k, v = case.inputs()
+    batch = _run(q, k, v, cu, "bf16")
+    for s in range(len(lens)):
+        a, b = cu[s], cu[s + 1]
+        alone = _run(q[a:b], k[a:b], v[a:b], np.array([0, b - a], np.int32), "bf16")
+        assert np.array_equal(alone, batch[a:b]), f"segment {s}"
+    order = [2, 0, 3, 1]
+    perm = lambda x: np.concatenate([x[cu[s]:cu[s + 1]] for s in order])
+    cu2 = workloads.cu_from_lengths([lens[s] for s in order])
+    out2 = _run(perm(q), perm(k), perm(v), cu2, "bf16")
+    assert np.array_equal(out2, perm(batch))
+
+
+def test_deterministic():
+    case = workloads.varlen8_case()
+    q, k, v = case.inputs()
+    a = _run(q, k, v, case.cu_seqlens, "bf16")
+    b = _run(q, k, v, case.cu_seqlens, "bf16")
+    assert np.array_equal(a, b)
+
+
+def test_long_single_segment():
+    """One 65536-token segment (4x the tower's full layer): sampled rows."""
+    case = workloads.Case("long65536", workloads.cu_from_lengths([65536]), seed=10, dtype="bf16")
+    _sampled_case(case, n_rows=256)
+
+
+def test_empty_inputs_are_noops():
+    import flash_attention_varlen_b200 as fa
+    z = torch.zeros(0, 16, 96, dtype=torch.bfloat16, device="cuda")
+    out = fa.attn_fwd(z, z, z, torch.zeros(1, dtype=torch.int32, device="cuda"))
+    assert out.shape == (0, 16, 96)
+    out = fa.attn_fwd(z, z, z, torch.zeros(4, dtype=torch.int32, device="cuda"))
+    assert out.shape == (0, 16, 96)
+
+
+def test_bad_seqlens_detected_on_device():
+    import flash_attention_varlen_b200 as fa
+    T = 300
+    q = torch.randn(T, 16, 96, device="cuda").to(torch.bfloat16)
+    out = torch.full_like(q, 7.0)
+    for bad in ([0, 200, 100, 300], [5, 300], [0, 299]):
+        cu = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        fa.attn_fwd(q, q, q, cu, out=out)          # host cannot see device data: queued
+        with pytest.raises(fa.VtAttnError) as e:
+            fa.check_device_status()
+        assert e.value.status == fa._binding.VT_ERR_BAD_SEQLENS
+        assert torch.all(out == 7.0)               # nothing written
+    good = torch.tensor([0, T], dtype=torch.int32, device="cuda")
+    fa.attn_fwd(q, q, q, good, out=out)
+    fa.check_device_status()
+    assert not torch.all(out == 7.0)
+
+
+def test_python_wrapper_validation():
+    import flash_attention_varlen_b200 as fa
+    q = torch.zeros(8, 16, 96, dtype=torch.bfloat16, device="cuda")
+    cu = torch.tensor([0, 8], dtype=torch.int32, device="cuda")
+    with pytest.raises(TypeError):
+        fa.attn_fwd(q, q, q.float(), cu)
+    with pytest.raises(TypeError):
+        fa.attn_fwd(q, q, q, cu.long())
+    with pytest.raises(fa.VtAttnError):
+        fa.attn_fwd(q[:, :, :64].contiguous(), q[:, :, :64].contiguous(),
+                    q[:, :, :64].contiguous(), cu)
+
+
+def test_host_buffers_end_to_end():
+    import flash_attention_varlen_b200 as fa
+    case = workloads.image896_cases()[0]
+    q, k, v = case.inputs()
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    cu = torch.from_numpy(case.cu_seqlens.copy())
+    fa.attn_fwd_host(pin(q), pin(k), pin(v), cu, out)
+    torch.cuda.synchronize()
+    got = out.float().numpy().astype(np.float64)
+    ref = _run(q, k, v, case.cu_seqlens, "bf16")
+    assert np.array_equal(got, ref)
