@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time budget of the oracle sample")
+    ap.add_argument("--single-layer", choices=["full", "window"], default=None,
+                    help="profiling aid: run only one tower layer (full = 1 x 16384 tok, "
+                         "window = 16 x 1024 tok) warmup + steps times and print its timing")
     return ap.parse_args(argv)
 
 
@@ -446,9 +449,39 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_single_layer(args):
+    """One layer type of the tower, called warmup + steps times (for ncu captures)."""
+    import torch
+    import flash_attention_varlen_b200 as fa
+    layer = 3 if args.single_layer == "full" else 0
+    case = workloads.tower_layer_case(layer, GRID)
+    q, k, v = case.inputs()
+    dev = torch.device("cuda", 0)
+    to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    dq, dk, dv = to(q), to(k), to(v)
+    out = torch.empty_like(dq)
+    cu = torch.from_numpy(case.cu_seqlens.copy()).to(dev)
+    for _ in range(args.warmup):
+        fa.attn_fwd(dq, dk, dv, cu, scale=SCALE, out=out)
+    fa.check_device_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fa.attn_fwd(dq, dk, dv, cu, scale=SCALE, out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    fa.check_device_status()
+    ms = e0.elapsed_time(e1) / max(1, args.steps)
+    print(json.dumps({"single_layer": args.single_layer, "ms_per_call": round(ms, 4),
+                      "tflops": round(case.flops() / (ms * 1e-3) / 1e12, 2),
+                      "calls": args.steps, "note": "back-to-back calls on one layer's inputs"}))
+
+
 def main(argv=None):
     args = parse_args(argv)
-    if args.impl == "reference":
+    if args.single_layer:
+        run_single_layer(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

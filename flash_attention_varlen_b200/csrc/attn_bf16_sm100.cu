@@ -9,22 +9,30 @@
 // One CTA (persistent, one per SM) works through units of 256 query rows of
 // one (segment, head): two 128-row Q tiles that share every K/V tile.
 //
+//   warps 8-11         : warp 8 loads, warp 9 issues MMAs, 10-11 idle (register donors)
 //   warp 8  (loader)   : TMA loads Q0/Q1 once per unit and K/V tiles into a
 //                        3-stage ring (64-byte swizzled, 32-column chunks).
 //   warp 9  (MMA)      : one thread issues tcgen05.mma:
 //                          S_i = Q_i K_j^T     (SS, M128 N128 K96)  -> TMEM
-//                          O_i += P_i V_j      (TS, M128 N96 K128; P read from TMEM)
+//                          O_i += P_i [V_j | 1] (TS, M128 N112 K128; P read from TMEM)
 //                        in the order S0 S1 | PV0 S0' | PV1 S1' | ... so that the
 //                        tensor core works on one tile while the other is in softmax.
 //   warps 0-3, 4-7     : softmax warpgroups for Q0 and Q1, one thread per row:
-//                        tcgen05.ld of the S row, row max, p = 2^(s*c - m) with a
+//                        tcgen05.ld of the S row, row max (three-input max tree),
+//                        p = 2^(s*c - m) (packed f32x2 FMA, then MUFU ex2) with a
 //                        deferred rescale (the running max m only moves when the
-//                        new tile max exceeds it by more than 8 in log2 units, so
-//                        O in TMEM is rarely touched), P packed to bf16 and written
-//                        back over S in TMEM, then the epilogue O / l -> bf16 -> HBM.
+//                        new tile max exceeds it by more than a threshold, so O in
+//                        TMEM is rarely touched), P packed to bf16 and written back
+//                        over S in TMEM, then the epilogue O / l -> bf16 -> HBM.
 //
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,352), O1 [384,480);
-// P_i overlays the first 64 columns of S_i (two bf16 per 32-bit column).
+// The row sum l is not accumulated by the softmax threads: each V stage carries
+// a fourth 32-column chunk whose first column is all ones, so column 96 of O
+// accumulates sum_j P_ij on the tensor core -- exactly the bf16-rounded weights
+// the PV product used -- and is rescaled together with O.
+//
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,368), O1 [384,496)
+// (O column 96 = l); P_i overlays the first 64 columns of S_i (two bf16 per
+// 32-bit column).
 //
 // Keys past the end of a segment inside its last tile are masked (p = 0);
 // query rows past the end are computed but not stored.  Every mbarrier wait is
@@ -39,21 +47,33 @@ constexpr int kBM = 128;          // query rows per Q tile
 constexpr int kBN = 128;          // keys per K/V tile
 constexpr int kD = 96;            // head width
 constexpr int kStages = 3;        // K/V ring depth
-constexpr int kTileBytes = kBM * kD * 2;   // 24576 (also a 128-key K or V tile)
+constexpr int kDv = kD + 16;               // PV N: 96 value columns + ones column (+15 zero)
+constexpr int kTileBytes = kBM * kD * 2;   // 24576: a 128-row Q or K tile
 constexpr int kChunkBytes = 128 * 64;      // 8192: 128 rows x 32 bf16
-constexpr int kThreads = 320;
+constexpr int kVTileBytes = 4 * kChunkBytes;  // V tile + the ones chunk
+constexpr int kThreads = 384;               // three warpgroups
+// Registers: launched at 168 per thread (65536 / 384, rounded down to 8); the two
+// softmax warpgroups raise theirs to 224 and the loader/MMA warpgroup drops to 56:
+// 2*128*224 + 128*56 = 64512 = 384*168, so the increase always finds its registers.
+constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 104;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "register split");
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: p stays below 2^8 between rescales
+// The running max only moves when a tile's max exceeds it by more than this (log2
+// units), so P stays below 2^3 between rescales.  Larger values save O rescales but
+// let the dominant key's p be rounded to bf16 more often (its error does not cancel
+// for a peaked softmax); 3 keeps a peaked (Q x 4) 1024-token row inside 1e-2 while
+// random N(0,1) rows almost never rescale.
+constexpr float kRescaleThreshold = 3.0f;
 
 static_assert(kBf16BlockRows == 2 * kBM, "a unit is two Q tiles");
 
 struct Smem {
   uint8_t q[2][kTileBytes];
   uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
+  uint8_t v[kStages][kVTileBytes];
   uint64_t q_full[2];
   uint64_t q_empty;
   uint64_t k_full[kStages];
@@ -101,8 +121,9 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t
   }
 }
 
-// O (+)= P V: P (128 x 128 bf16) from TMEM, V MN-major (head dim contiguous):
-// 8-key groups 512 B apart (SBO), 32-column chunks 8 KB apart (LBO); eight K16 steps.
+// O (+)= P [V | 1]: P (128 x 128 bf16) from TMEM, V MN-major (head dim contiguous):
+// 8-key groups 512 B apart (SBO), 32-column chunks 8 KB apart (LBO), N = 112 reaching
+// into the ones chunk; eight K16 steps.
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_s,
                                          uint32_t idesc, bool accumulate) {
 #pragma unroll
@@ -157,6 +178,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.abort_flag = 0;
     fence_mbar_init();
   }
+  // Ones chunk of every V stage: row r holds bf16 1.0 in column 0 and zeros elsewhere,
+  // in the 64-byte swizzle the MMA reads (16-byte unit u of row r is stored at unit
+  // u ^ ((r >> 1) & 3)).  TMA never writes this chunk.
+  for (int i = tid; i < kStages * 128 * 4; i += kThreads) {
+    const int st = i / (128 * 4), r = (i / 4) % 128, unit = i % 4;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (unit == ((r >> 1) & 3)) val.x = 0x3F80u;  // bf16 1.0 in the low half = column 0
+    *reinterpret_cast<uint4*>(sm.v[st] + 3 * kChunkBytes + r * 64 + unit * 16) = val;
+  }
+  fence_proxy_async_smem();
   if (warp == kWarpMma) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -173,7 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &sm.abort_flag;
   int* dev_status = a.dev_status;
 
-  if (warp == kWarpLoad) {
+  if (warp >= 8) {
+   setmaxnreg_dec<kRegsOther>();
+   if (warp == kWarpLoad) {
     // ------------------------------------------------------------ loader
     if (lane == 0) {
       uint32_t kv_it = 0, unit_it = 0, q0_loads = 0, q1_loads = 0, k_issued = 0, v_issued = 0;
@@ -221,11 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait_drain(&sm.v_full[f % kStages], (f / kStages) & 1);
       }
     }
-  } else if (warp == kWarpMma) {
+   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = a.idesc_qk;
-      const uint32_t idesc_pv = make_idesc_bf16(kBM, kD, false, true, false);
+      const uint32_t idesc_pv = make_idesc_bf16(kBM, kDv, false, true, false);
       const uint32_t q_s0 = smem_u32(sm.q[0]), q_s1 = smem_u32(sm.q[1]);
       uint32_t kv_it = 0, unit_it = 0, q1_it = 0, p_cnt0 = 0, p_cnt1 = 0;
       for (long long u = blockIdx.x; u < total; u += gridDim.x, ++unit_it) {
@@ -289,8 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&sm.drain);
       mbar_wait_drain(&sm.drain, 0);
     }
+   }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
+    setmaxnreg_inc<kRegsSoftmax>();
     const int wg = warp >> 2;
     const int r = tid & 127;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -302,29 +337,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit x = decode_unit(u, E, a.entries, a.cu_seqlens);
       if (wg == 1 && !x.has_q1) continue;
       const int row_tok = x.q0 + wg * kBM + r;
-      float m = 0.f, l = 0.f;
+      float m = 0.f;
       bool ok = true;
       for (int j = 0; j < x.nkv; ++j) {
         if (!warp_wait(&sm.s_full[wg], s_cnt & 1, abort_flag, dev_status)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
-        uint32_t s[kBN];
-        tmem_ld32(tS + 0, s);
-        tmem_ld32(tS + 32, s + 32);
-        tmem_ld32(tS + 64, s + 64);
-        tmem_ld32(tS + 96, s + 96);
+        uint32_t su[kBN];
+        tmem_ld32(tS + 0, su);
+        tmem_ld32(tS + 32, su + 32);
+        tmem_ld32(tS + 64, su + 64);
+        tmem_ld32(tS + 96, su + 96);
         tmem_ld_wait();
-        reg_fence<kBN>(s);
+        reg_fence<kBN>(su);
+        float* sf = reinterpret_cast<float*>(su);
         const int nvalid = x.seg_end - (x.seg_start + j * kBN);  // >= 1
-        float mx = -INFINITY;
-        if (nvalid >= kBN) {
-#pragma unroll
-          for (int i = 0; i < kBN; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
-        } else {
+        const bool masked = nvalid < kBN;
+        if (masked) {
 #pragma unroll
           for (int i = 0; i < kBN; ++i)
-            if (i < nvalid) mx = fmaxf(mx, __uint_as_float(s[i]));
+            if (i >= nvalid) sf[i] = -INFINITY;
         }
+        // row max: eight independent three-input max chains
+        float pm[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) pm[q] = fmaxf(sf[q], sf[q + 8]);
+#pragma unroll
+        for (int i = 16; i < kBN; i += 16) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) pm[q] = fmax3(pm[q], sf[i + q], sf[i + 8 + q]);
+        }
+        const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]),
+                               fmaxf(pm[6], pm[7]));
         const float mt = mx * c;
         float alpha = 1.f;
         bool rescale = false;
@@ -335,45 +379,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = mt;
           rescale = true;
         }
-        const float neg_m = -m;
-        float sum0 = 0.f, sum1 = 0.f;
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
         uint32_t p[kBN / 2];
-        if (nvalid >= kBN) {
+#pragma unroll
+        for (int i = 0; i < kBN / 2; ++i) {
+          const float2 t = ffma2(make_float2(sf[2 * i], sf[2 * i + 1]), c2, nm2);
+          p[i] = pack_bf16x2(ex2_approx(t.x), ex2_approx(t.y));
+        }
+        if (masked) {  // exact zeros past the segment end (also when scale is 0)
 #pragma unroll
           for (int i = 0; i < kBN / 2; ++i) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * i]), c, neg_m));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * i + 1]), c, neg_m));
-            sum0 += p0;
-            sum1 += p1;
-            p[i] = pack_bf16x2(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < kBN / 2; ++i) {
-            const float p0 = (2 * i < nvalid) ? ex2_approx(fmaf(__uint_as_float(s[2 * i]), c, neg_m)) : 0.f;
-            const float p1 = (2 * i + 1 < nvalid) ? ex2_approx(fmaf(__uint_as_float(s[2 * i + 1]), c, neg_m)) : 0.f;
-            sum0 += p0;
-            sum1 += p1;
-            p[i] = pack_bf16x2(p0, p1);
+            if (2 * i >= nvalid) p[i] = 0u;
+            else if (2 * i + 1 >= nvalid) p[i] &= 0xFFFFu;
           }
         }
-        l = l * alpha + (sum0 + sum1);
         if (__any_sync(0xffffffffu, rescale)) {
-          // O must hold PV_{j-1} before it is scaled (the commit behind S_j already
-          // implies it; the wait makes it explicit).
+          // O (with its row-sum column) must hold PV_{j-1} before it is scaled (the commit
+          // behind S_j already implies it; the wait makes it explicit).
           if (!warp_wait(&sm.o_done[wg], (o_base + j - 1) & 1, abort_flag, dev_status)) { ok = false; break; }
           tc_fence_after();
-          uint32_t o[kD];
+          uint32_t o[kDv];
           tmem_ld32(tO + 0, o);
           tmem_ld32(tO + 32, o + 32);
           tmem_ld32(tO + 64, o + 64);
+          tmem_ld16(tO + 96, o + 96);
           tmem_ld_wait();
-          reg_fence<kD>(o);
+          reg_fence<kDv>(o);
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-          for (int i = 0; i < kD; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < kDv; i += 2) {
+            const float2 y = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+            o[i] = __float_as_uint(y.x);
+            o[i + 1] = __float_as_uint(y.y);
+          }
           tmem_st32(tO + 0, o);
           tmem_st32(tO + 32, o + 32);
           tmem_st32(tO + 64, o + 64);
+          tmem_st16(tO + 96, o + 96);
         }
         tmem_st32(tS + 0, p);
         tmem_st32(tS + 32, p + 32);
@@ -382,27 +424,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.p_full[wg]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 -> HBM (rows inside the segment only)
+      // epilogue: O / l -> bf16 -> HBM (rows inside the segment only); l = O column 96
       if (!warp_wait(&sm.o_done[wg], (o_base + x.nkv - 1) & 1, abort_flag, dev_status)) break;
       tc_fence_after();
-      uint32_t o[kD];
+      uint32_t o[kD + 1];
       tmem_ld32(tO + 0, o);
       tmem_ld32(tO + 32, o + 32);
       tmem_ld32(tO + 64, o + 64);
+      tmem_ld1(tO + 96, o[96]);
       tmem_ld_wait();
-      reg_fence<kD>(o);
+      reg_fence<kD + 1>(o);
       if (row_tok < x.seg_end) {
-        const float inv_l = 1.0f / l;
+        const float inv_l = 1.0f / __uint_as_float(o[96]);
         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) +
                                               (static_cast<size_t>(row_tok) * a.H + x.head) * (kD * 2));
+        const float2 il2 = make_float2(inv_l, inv_l);
 #pragma unroll
         for (int i = 0; i < kD / 8; ++i) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
-          w.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
-          w.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
-          w.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
-          dst[i] = w;
+          uint32_t w[4];
+#pragma unroll
+          for (int h2 = 0; h2 < 4; ++h2) {
+            const float2 y = fmul2(make_float2(__uint_as_float(o[8 * i + 2 * h2]),
+                                               __uint_as_float(o[8 * i + 2 * h2 + 1])), il2);
+            w[h2] = pack_bf16x2(y.x, y.y);
+          }
+          dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       o_base += x.nkv;
