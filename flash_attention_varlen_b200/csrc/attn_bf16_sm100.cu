@@ -67,6 +67,10 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 // for a peaked softmax); 3 keeps a peaked (Q x 4) 1024-token row inside 1e-2 while
 // random N(0,1) rows almost never rescale.
 constexpr float kRescaleThreshold = 3.0f;
+// Every kPolyEvery-th pair of scores takes its exp2 on the FMA pipe (polynomial)
+// instead of the MUFU, which is otherwise the busiest unit (one exp2 per 384
+// tensor FLOPs at head width 96).  0 disables.
+constexpr int kPolyEvery = 0;
 
 static_assert(kBf16BlockRows == 2 * kBM, "a unit is two Q tiles");
 
@@ -81,7 +85,7 @@ struct Smem {
   uint64_t v_full[kStages];
   uint64_t v_empty[kStages];
   uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t p_full[2][2];  // [Q tile][key half]: P columns 0-31 / 32-63 written
   uint64_t o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -109,27 +113,41 @@ __device__ __forceinline__ Unit decode_unit(long long u, int E, const WorkEntry*
   return x;
 }
 
+// The MMA thread shares its SM sub-partition with softmax warps that issue every
+// cycle, so it must spend as few instructions per MMA as possible: descriptors are
+// built once per tile base and each K16 step only adds a constant to the start
+// address field (16-byte units; never carries out of the 14-bit field since
+// shared addresses stay below 256 KB).
+
 // S = Q K^T: both operands K-major (head dim contiguous), 64-byte swizzle,
 // three 32-column chunks of 8 KB; K = 96 as six K16 steps.
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t k_s,
+__device__ __forceinline__ uint64_t qk_desc(uint32_t saddr) {
+  return make_smem_desc(saddr, 16, 512, kSwizzle64B);
+}
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc,
                                          uint32_t idesc) {
 #pragma unroll
   for (int kk = 0; kk < kD / 16; ++kk) {
-    const uint32_t off = (kk >> 1) * kChunkBytes + (kk & 1) * 32;
-    mma_ss(d_tmem, make_smem_desc(q_s + off, 16, 512, kSwizzle64B),
-           make_smem_desc(k_s + off, 16, 512, kSwizzle64B), idesc, kk > 0 ? 1u : 0u);
+    const uint64_t off = static_cast<uint64_t>(((kk >> 1) * kChunkBytes + (kk & 1) * 32) >> 4);
+    mma_ss(d_tmem, q_desc + off, k_desc + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 // O (+)= P [V | 1]: P (128 x 128 bf16) from TMEM, V MN-major (head dim contiguous):
 // 8-key groups 512 B apart (SBO), 32-column chunks 8 KB apart (LBO), N = 112 reaching
 // into the ones chunk; eight K16 steps.
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_s,
-                                         uint32_t idesc, bool accumulate) {
+__device__ __forceinline__ uint64_t pv_desc(uint32_t saddr) {
+  return make_smem_desc(saddr, kChunkBytes, 512, kSwizzle64B);
+}
+// One half of the K loop (keys 64*half .. +63), so the product can start on the
+// first 64 keys while the softmax still computes the other 64.
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
+                                              uint32_t idesc, int half, bool accumulate) {
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk) {
-    mma_ts(d_tmem, p_tmem + kk * 8, make_smem_desc(v_s + kk * 1024, kChunkBytes, 512, kSwizzle64B),
-           idesc, (accumulate || kk > 0) ? 1u : 0u);
+  for (int k4 = 0; k4 < kBN / 32; ++k4) {
+    const int kk = half * (kBN / 32) + k4;
+    mma_ts(d_tmem, p_tmem + kk * 8, v_desc + static_cast<uint64_t>((kk * 1024) >> 4), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -164,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], kBM);
+      mbar_init(&sm.p_full[i][0], kBM);
+      mbar_init(&sm.p_full[i][1], kBM);
       mbar_init(&sm.o_done[i], 1);
     }
     mbar_init(&sm.q_empty, 1);
@@ -259,7 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = a.idesc_qk;
       const uint32_t idesc_pv = make_idesc_bf16(kBM, kDv, false, true, false);
-      const uint32_t q_s0 = smem_u32(sm.q[0]), q_s1 = smem_u32(sm.q[1]);
+      const uint64_t dq0 = qk_desc(smem_u32(sm.q[0])), dq1 = qk_desc(smem_u32(sm.q[1]));
+      // stage s of the K (V) ring starts kTileBytes (kVTileBytes) after stage s-1
+      const uint64_t dk0 = qk_desc(smem_u32(sm.k[0])), dv0 = pv_desc(smem_u32(sm.v[0]));
+      auto dk = [&](uint32_t st) { return dk0 + static_cast<uint64_t>(st * (kTileBytes >> 4)); };
+      auto dv = [&](uint32_t st) { return dv0 + static_cast<uint64_t>(st * (kVTileBytes >> 4)); };
       uint32_t kv_it = 0, unit_it = 0, q1_it = 0, p_cnt0 = 0, p_cnt1 = 0;
       for (long long u = blockIdx.x; u < total; u += gridDim.x, ++unit_it) {
         const Unit x = decode_unit(u, E, a.entries, a.cu_seqlens);
@@ -270,11 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = kv_it % kStages;
           if (!mbar_wait_bounded(&sm.k_full[st], (kv_it / kStages) & 1, abort_flag, dev_status)) break;
           tc_fence_after();
-          const uint32_t k_s = smem_u32(sm.k[st]);
-          issue_qk(tmem + kColS0, q_s0, k_s, idesc_qk);
+          issue_qk(tmem + kColS0, dq0, dk(st), idesc_qk);
           mma_commit(&sm.s_full[0]);
           if (x.has_q1) {
-            issue_qk(tmem + kColS1, q_s1, k_s, idesc_qk);
+            issue_qk(tmem + kColS1, dq1, dk(st), idesc_qk);
             mma_commit(&sm.s_full[1]);
           }
           mma_commit(&sm.k_empty[st]);
@@ -284,27 +306,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t it = kv_it + j, st = it % kStages;
           const bool more = j + 1 < x.nkv;
           const uint32_t st1 = (it + 1) % kStages;
-          const uint32_t v_s = smem_u32(sm.v[st]);
-          if (!mbar_wait_bounded(&sm.p_full[0], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
-          ++p_cnt0;
           if (!mbar_wait_bounded(&sm.v_full[st], (it / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
+          if (!mbar_wait_bounded(&sm.p_full[0][0], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(tmem + kColO0, tmem + kColS0, v_s, idesc_pv, j > 0);
+          issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 0, j > 0);
+          if (!mbar_wait_bounded(&sm.p_full[0][1], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
+          ++p_cnt0;
+          tc_fence_after();
+          issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 1, true);
           mma_commit(&sm.o_done[0]);
           if (more) {
             if (!mbar_wait_bounded(&sm.k_full[st1], ((it + 1) / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
             tc_fence_after();
-            issue_qk(tmem + kColS0, q_s0, smem_u32(sm.k[st1]), idesc_qk);
+            issue_qk(tmem + kColS0, dq0, dk(st1), idesc_qk);
             mma_commit(&sm.s_full[0]);
           }
           if (x.has_q1) {
-            if (!mbar_wait_bounded(&sm.p_full[1], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
+            if (!mbar_wait_bounded(&sm.p_full[1][0], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 0, j > 0);
+            if (!mbar_wait_bounded(&sm.p_full[1][1], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
             ++p_cnt1;
             tc_fence_after();
-            issue_pv(tmem + kColO1, tmem + kColS1, v_s, idesc_pv, j > 0);
+            issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 1, true);
             mma_commit(&sm.o_done[1]);
             if (more) {
-              issue_qk(tmem + kColS1, q_s1, smem_u32(sm.k[st1]), idesc_qk);
+              issue_qk(tmem + kColS1, dq1, dk(st1), idesc_qk);
               mma_commit(&sm.s_full[1]);
             }
           }
@@ -343,29 +370,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!warp_wait(&sm.s_full[wg], s_cnt & 1, abort_flag, dev_status)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
-        uint32_t su[kBN];
-        tmem_ld32(tS + 0, su);
-        tmem_ld32(tS + 32, su + 32);
-        tmem_ld32(tS + 64, su + 64);
-        tmem_ld32(tS + 96, su + 96);
-        tmem_ld_wait();
-        reg_fence<kBN>(su);
-        float* sf = reinterpret_cast<float*>(su);
         const int nvalid = x.seg_end - (x.seg_start + j * kBN);  // >= 1
         const bool masked = nvalid < kBN;
-        if (masked) {
-#pragma unroll
-          for (int i = 0; i < kBN; ++i)
-            if (i >= nvalid) sf[i] = -INFINITY;
-        }
-        // row max: eight independent three-input max chains
+        // pass 1, row max: the row in two 64-column halves, eight independent
+        // three-input max chains
         float pm[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) pm[q] = fmaxf(sf[q], sf[q + 8]);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t su[kBN / 2];
+          float* sf = reinterpret_cast<float*>(su);
+          tmem_ld32(tS + half * 64, su);
+          tmem_ld32(tS + half * 64 + 32, su + 32);
+          tmem_ld_wait();
+          reg_fence<kBN / 2>(su);
+          if (masked) {
 #pragma unroll
-        for (int i = 16; i < kBN; i += 16) {
+            for (int i = 0; i < kBN / 2; ++i)
+              if (half * 64 + i >= nvalid) sf[i] = -INFINITY;
+          }
+          if (half == 0) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) pm[q] = fmax3(pm[q], sf[i + q], sf[i + 8 + q]);
+            for (int q = 0; q < 8; ++q) pm[q] = fmaxf(sf[q], sf[q + 8]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) pm[q] = fmax3(pm[q], sf[q], sf[q + 8]);
+          }
+#pragma unroll
+          for (int i = 16; i < kBN / 2; i += 16) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) pm[q] = fmax3(pm[q], sf[i + q], sf[i + 8 + q]);
+          }
         }
         const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]),
                                fmaxf(pm[6], pm[7]));
@@ -379,49 +413,68 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = mt;
           rescale = true;
         }
-        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
-        uint32_t p[kBN / 2];
-#pragma unroll
-        for (int i = 0; i < kBN / 2; ++i) {
-          const float2 t = ffma2(make_float2(sf[2 * i], sf[2 * i + 1]), c2, nm2);
-          p[i] = pack_bf16x2(ex2_approx(t.x), ex2_approx(t.y));
-        }
-        if (masked) {  // exact zeros past the segment end (also when scale is 0)
-#pragma unroll
-          for (int i = 0; i < kBN / 2; ++i) {
-            if (2 * i >= nvalid) p[i] = 0u;
-            else if (2 * i + 1 >= nvalid) p[i] &= 0xFFFFu;
-          }
-        }
         if (__any_sync(0xffffffffu, rescale)) {
           // O (with its row-sum column) must hold PV_{j-1} before it is scaled (the commit
           // behind S_j already implies it; the wait makes it explicit).
           if (!warp_wait(&sm.o_done[wg], (o_base + j - 1) & 1, abort_flag, dev_status)) { ok = false; break; }
           tc_fence_after();
-          uint32_t o[kDv];
-          tmem_ld32(tO + 0, o);
-          tmem_ld32(tO + 32, o + 32);
-          tmem_ld32(tO + 64, o + 64);
-          tmem_ld16(tO + 96, o + 96);
-          tmem_ld_wait();
-          reg_fence<kDv>(o);
+          // in 32-column chunks to keep the register footprint small
           const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-          for (int i = 0; i < kDv; i += 2) {
-            const float2 y = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
-            o[i] = __float_as_uint(y.x);
-            o[i + 1] = __float_as_uint(y.y);
+          for (int c0 = 0; c0 < kDv; c0 += 32) {
+            uint32_t o[32];
+            if (c0 + 32 <= kDv) tmem_ld32(tO + c0, o);
+            else tmem_ld16(tO + c0, o);
+            tmem_ld_wait();
+            reg_fence<32>(o);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 y = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+              o[i] = __float_as_uint(y.x);
+              o[i + 1] = __float_as_uint(y.y);
+            }
+            if (c0 + 32 <= kDv) tmem_st32(tO + c0, o);
+            else tmem_st16(tO + c0, o);
           }
-          tmem_st32(tO + 0, o);
-          tmem_st32(tO + 32, o + 32);
-          tmem_st32(tO + 64, o + 64);
-          tmem_st16(tO + 96, o + 96);
         }
-        tmem_st32(tS + 0, p);
-        tmem_st32(tS + 32, p + 32);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&sm.p_full[wg]);
+        // P in two key halves: the PV product of the first 64 keys starts while the
+        // exponentials of the other 64 are computed
+        // pass 2: reload each half of S, exponentiate, store its P half (P half 0
+        // overwrites S columns 0-31 only after that half has been read)
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t su[kBN / 2];
+          const float* sf = reinterpret_cast<const float*>(su);
+          tmem_ld32(tS + half * 64, su);
+          tmem_ld32(tS + half * 64 + 32, su + 32);
+          tmem_ld_wait();
+          reg_fence<kBN / 2>(su);
+          uint32_t p[kBN / 4];
+#pragma unroll
+          for (int i2 = 0; i2 < kBN / 4; ++i2) {
+            const int i = half * (kBN / 4) + i2;
+            const float2 t = ffma2(make_float2(sf[2 * i2], sf[2 * i2 + 1]), c2, nm2);
+            if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
+              const float2 e = exp2_poly2(t);  // FMA pipe: takes load off the MUFU
+              p[i2] = pack_bf16x2(e.x, e.y);
+            } else {
+              p[i2] = pack_bf16x2(ex2_approx(t.x), ex2_approx(t.y));
+            }
+          }
+          if (masked) {  // exact zeros past the segment end (also when scale is 0)
+#pragma unroll
+            for (int i2 = 0; i2 < kBN / 4; ++i2) {
+              const int i = half * (kBN / 4) + i2;
+              if (2 * i >= nvalid) p[i2] = 0u;
+              else if (2 * i + 1 >= nvalid) p[i2] &= 0xFFFFu;
+            }
+          }
+          tmem_st32(tS + half * (kBN / 4), p);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&sm.p_full[wg][half]);
+        }
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 -> HBM (rows inside the segment only); l = O column 96

@@ -295,6 +295,38 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return d;
 }
 
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for a pair, on the FMA/ALU pipes instead of the MUFU (Cody-Waite range
+// reduction + minimax polynomial): x = n + f with n = rint(x) found by the
+// 1.5 * 2^23 shift and f in [-1/2, 1/2]; 2^f ~ c0 + f (c1 + f (c2 + f c3)), the
+// degree-3 polynomial minimising the maximum relative error on [-1/2, 1/2]
+// (Remez exchange, fit_exp2_poly.py: 7.5e-5); 2^n enters by adding n to the
+// exponent field.  x is clamped at -127 (results below 2^-127 are not needed:
+// every row holds a 1 at its running max).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
+  const float2 shift = make_float2(12582912.0f, 12582912.0f);
+  const float2 xi = fadd2(x, shift);
+  const float2 n = fadd2(xi, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = ffma2(f, make_float2(0x1.c3f76p-5f, 0x1.c3f76p-5f),
+                   make_float2(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+  p = ffma2(p, f, make_float2(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+  p = ffma2(p, f, make_float2(0x1.fff692p-1f, 0x1.fff692p-1f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(xi.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(xi.y) << 23)));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
