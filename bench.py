@@ -72,6 +72,16 @@ def rank_base_seed(rank: int) -> int:
     return 1000 * rank
 
 
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """Max of a per-rank float over the process group (identity when not distributed)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -272,9 +282,7 @@ def run_ours(args):
     fa.check_device_status(stream)
     total_ms = t_start.elapsed_time(t_end)
     if distributed:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, dist, dev)
         dist.barrier()
 
     per_layer = np.array([[ev[s][l][0].elapsed_time(ev[s][l][1]) for l in range(n_layers)]
@@ -393,11 +401,7 @@ def run_e2e(fa, torch, dev, pinned, cases, steps, step_flops, world, dist):
     ev1.record(streams[0])
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - t0
-    ms = ev0.elapsed_time(ev1)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
     h2d = sum(3 * T * H * D * 2 + (c.num_segments + 1) * 4 for c in cases)
     d2h = len(cases) * T * H * D * 2
     return {"value": round(step_flops * steps * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
