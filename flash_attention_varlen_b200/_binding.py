@@ -45,7 +45,7 @@ def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"libvtattn.so not found at {LIB_PATH}; build it with "
-            "`python -m flash_attention_varlen_b200.build` (nvcc, sm_100a). "
+            "`python flash_attention_varlen_b200/build.py` (nvcc, sm_100a). "
             "There is no CPU fallback.")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float

@@ -1,6 +1,8 @@
 """Builds libvtattn.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m flash_attention_varlen_b200.build [--force] [--verbose]
+    python flash_attention_varlen_b200/build.py [--force] [--verbose]
+
+Run it as a script (or load it by path): importing the package loads the library.
 """
 from __future__ import annotations
 

@@ -16,8 +16,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def binding():
-    from flash_attention_varlen_b200 import build as b
-    b.build()
+    from conftest import build_cuda_library
+    build_cuda_library()
     from flash_attention_varlen_b200 import _binding
     return _binding
 

@@ -29,8 +29,8 @@ SCALE = 1.0 / math.sqrt(96)
 def _need_gpu():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    from flash_attention_varlen_b200 import build
-    build.build()
+    from conftest import build_cuda_library
+    build_cuda_library()
 
 
 def _to_dev(a, dtype):
