@@ -26,6 +26,7 @@ VT_ERR_DEVICE_TIMEOUT = 6
 # every symbol include/vt_attn.h declares
 EXPORTED = (
     "vt_attn_fwd",
+    "vt_attn_fwd_noalloc",
     "vt_attn_validate_seqlens_host",
     "vt_attn_smem_bytes",
     "vt_attn_workspace_bytes",
@@ -51,6 +52,8 @@ def _load():
     P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
     lib.vt_attn_fwd.argtypes = [P, P, P, P, P, I32, I32, I32, I32, F, ctypes.c_int, P]
     lib.vt_attn_fwd.restype = ctypes.c_int
+    lib.vt_attn_fwd_noalloc.argtypes = lib.vt_attn_fwd.argtypes
+    lib.vt_attn_fwd_noalloc.restype = ctypes.c_int
     lib.vt_attn_validate_seqlens_host.argtypes = [P, I32, I32]
     lib.vt_attn_validate_seqlens_host.restype = ctypes.c_int
     lib.vt_attn_smem_bytes.argtypes = [I32, ctypes.c_int]
@@ -74,6 +77,15 @@ def vt_attn_fwd(q: int, k: int, v: int, out: int, cu_seqlens: int, num_segments:
     """Raw entry point: device pointers as ints; returns the vt_status code."""
     return lib.vt_attn_fwd(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D,
                            ctypes.c_float(scale), dtype, stream)
+
+
+def vt_attn_fwd_noalloc(q: int, k: int, v: int, out: int, cu_seqlens: int, num_segments: int,
+                        total_tokens: int, H: int, D: int, scale: float, dtype: int,
+                        stream: int) -> int:
+    """vt_attn_fwd for callers that cannot let the library allocate device memory
+    (fixed 1 MiB work-list array; see include/vt_attn.h for limits and sharing rules)."""
+    return lib.vt_attn_fwd_noalloc(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D,
+                                   ctypes.c_float(scale), dtype, stream)
 
 
 def vt_attn_validate_seqlens_host(cu_seqlens_host: int, num_segments: int, total_tokens: int) -> int:

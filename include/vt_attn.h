@@ -76,6 +76,36 @@ vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
                       int32_t H, int32_t D, float scale, vt_dtype dtype, void* stream);
 
 /*
+ * vt_attn_fwd without any device allocation by the library.  (The source pages
+ * have no counterpart to this entry point; it exists for callers, not for the
+ * method.)
+ *
+ * For callers that cannot let a library allocate device memory: programs whose
+ * device memory is owned entirely by their own allocator or pool, programs that
+ * must not incur the device-wide synchronisation cudaMalloc/cudaFree may cause,
+ * and programs that only allocate at start-up.  Arguments, layouts and results
+ * are those of vt_attn_fwd; the work list lives in a fixed 1 MiB array in the
+ * library's device memory (held on every GPU that loads the library until the
+ * process exits) instead of a per-stream allocation.
+ *
+ * Limits and rules:
+ *   - the work list must fit: 128 + 8 * (ceil(T / R) + num_segments) <= 1 MiB,
+ *     R = 256 for bf16, 64 for f32 (e.g. bf16 T = 16384 with 16 segments uses
+ *     768 bytes); larger calls return VT_ERR_UNSUPPORTED and launch nothing;
+ *   - the first call on a device looks up the array's device address for that
+ *     device (make it with the device current, before capturing the stream into
+ *     anything);
+ *   - every call on a device shares the array, so calls that may overlap on the
+ *     GPU (e.g. on two streams) race and must be serialised by the caller;
+ *   - a malformed cu_seqlens makes the call write nothing; it is not reported by
+ *     vt_attn_last_device_status, which covers vt_attn_fwd's own work lists.
+ */
+vt_status vt_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                              const int32_t* cu_seqlens, int32_t num_segments,
+                              int32_t total_tokens, int32_t H, int32_t D, float scale,
+                              vt_dtype dtype, void* stream);
+
+/*
  * Pure host check of a host copy of cu_seqlens (num_segments+1 entries):
  * VT_OK, VT_ERR_NULL or VT_ERR_BAD_SEQLENS.  Touches no GPU.
  */
