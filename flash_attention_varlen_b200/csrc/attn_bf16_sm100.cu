@@ -9,9 +9,11 @@
 // One CTA (persistent, one per SM) works through units of 256 query rows of
 // one (segment, head): two 128-row Q tiles that share every K/V tile.
 //
-//   warps 8-11         : warp 8 loads, warp 9 issues MMAs, 10-11 idle (register donors)
-//   warp 8  (loader)   : TMA loads Q0/Q1 once per unit and K/V tiles into a
-//                        3-stage ring (64-byte swizzled, 32-column chunks).
+//   warps 8-11         : warp 8 loads K/V, warp 9 issues MMAs, warp 10 loads Q, 11 idle
+//   warp 8  (K/V loader): TMA loads of K/V tiles into a 2-stage ring (64-byte
+//                        swizzled, 32-column chunks).
+//   warp 10 (Q loader) : TMA loads of Q0/Q1 into a double buffer, so the next
+//                        unit's Q arrives while the current unit still runs.
 //   warp 9  (MMA)      : one thread issues tcgen05.mma:
 //                          S_i = Q_i K_j^T     (SS, M128 N128 K96)  -> TMEM
 //                          O_i += P_i [V_j | 1] (TS, M128 N112 K128; P read from TMEM)
@@ -46,19 +48,21 @@ namespace {
 constexpr int kBM = 128;          // query rows per Q tile
 constexpr int kBN = 128;          // keys per K/V tile
 constexpr int kD = 96;            // head width
-constexpr int kStages = 3;        // K/V ring depth
+constexpr int kStages = 2;        // K/V ring depth
+constexpr int kQBufs = 2;         // Q is double-buffered: the next unit's Q lands during this one
 constexpr int kDv = kD + 16;               // PV N: 96 value columns + ones column (+15 zero)
 constexpr int kTileBytes = kBM * kD * 2;   // 24576: a 128-row Q or K tile
 constexpr int kChunkBytes = 128 * 64;      // 8192: 128 rows x 32 bf16
 constexpr int kVTileBytes = 4 * kChunkBytes;  // V tile + the ones chunk
 constexpr int kThreads = 384;               // three warpgroups
 // Registers: launched at 168 per thread (65536 / 384, rounded down to 8); the two
-// softmax warpgroups raise theirs to 224 and the loader/MMA warpgroup drops to 56:
-// 2*128*224 + 128*56 = 64512 = 384*168, so the increase always finds its registers.
-constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 104;
+// softmax warpgroups raise theirs to 192 and the loader/MMA warpgroup drops to 120:
+// 2*128*192 + 128*120 = 64512 = 384*168, so the increase always finds its registers.
+constexpr uint32_t kRegsSoftmax = 192, kRegsOther = 120;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "register split");
-constexpr int kWarpLoad = 8;
+constexpr int kWarpLoad = 8;       // K/V loader
 constexpr int kWarpMma = 9;
+constexpr int kWarpLoadQ = 10;     // Q loader (runs up to one unit ahead)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 // The running max only moves when a tile's max exceeds it by more than this (log2
@@ -75,11 +79,11 @@ constexpr int kPolyEvery = 0;
 static_assert(kBf16BlockRows == 2 * kBM, "a unit is two Q tiles");
 
 struct Smem {
-  uint8_t q[2][kTileBytes];
+  uint8_t q[kQBufs][2][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kVTileBytes];
-  uint64_t q_full[2];
-  uint64_t q_empty;
+  uint64_t q_full[kQBufs][2];
+  uint64_t q_empty[kQBufs];
   uint64_t k_full[kStages];
   uint64_t k_empty[kStages];
   uint64_t v_full[kStages];
@@ -99,18 +103,47 @@ struct Unit {
   bool has_q1;
 };
 
-__device__ __forceinline__ Unit decode_unit(long long u, int E, const WorkEntry* entries,
-                                            const int32_t* cu) {
-  Unit x;
-  const int e = static_cast<int>(u % E);
-  x.head = static_cast<int>(u / E);
-  const WorkEntry we = entries[e];
-  x.seg_start = cu[we.seg];
-  x.seg_end = cu[we.seg + 1];
-  x.q0 = x.seg_start + we.qblock * (2 * kBM);
-  x.has_q1 = x.q0 + kBM < x.seg_end;
-  x.nkv = (x.seg_end - x.seg_start + kBN - 1) / kBN;
-  return x;
+// Walks this CTA's units u = blockIdx.x, + gridDim.x, ... (unit u = head u / E,
+// entry u % E).  Each unit is decoded from its 16-byte entry, and the next unit's
+// entry is loaded as soon as the current one is taken, so the load's latency is
+// hidden behind a whole unit of work instead of stalling every role at each unit
+// boundary.  The total unit count stays below 2^31: it is bounded by the tokens x
+// heads that fit in device memory.
+class UnitStream {
+ public:
+  __device__ __forceinline__ UnitStream(const WorkEntry* entries, uint32_t E, uint32_t total)
+      : entries_(reinterpret_cast<const int4*>(entries)), E_(E), total_(total), u_(blockIdx.x) {
+    e_ = E ? u_ % E : 0;
+    head_ = E ? u_ / E : 0;
+    cur_ = u_ < total_ ? __ldg(entries_ + e_) : make_int4(0, 0, 0, 0);
+  }
+  __device__ __forceinline__ bool valid() const { return u_ < total_; }
+  __device__ __forceinline__ Unit take() {
+    Unit x;
+    x.head = static_cast<int>(head_);
+    x.seg_start = cur_.z;
+    x.seg_end = cur_.w;
+    x.q0 = x.seg_start + cur_.y * (2 * kBM);
+    x.has_q1 = x.q0 + kBM < x.seg_end;
+    x.nkv = (x.seg_end - x.seg_start + kBN - 1) / kBN;
+    e_ += gridDim.x;
+    head_ += e_ / E_;
+    e_ %= E_;
+    u_ += gridDim.x;
+    if (u_ < total_) cur_ = __ldg(entries_ + e_);
+    return x;
+  }
+
+ private:
+  const int4* entries_;
+  uint32_t E_, total_, u_, e_, head_;
+  int4 cur_;
+};
+
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 // The MMA thread shares its SM sub-partition with softmax warps that issue every
@@ -174,19 +207,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (raw & 1023u)) & 1023u));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int E = a.hdr->num_entries;
-  const long long total = static_cast<long long>(E) * a.H;
-  if (static_cast<long long>(blockIdx.x) >= total) return;  // uniform over the CTA
+  const uint32_t E = static_cast<uint32_t>(a.hdr->num_entries);
+  const uint32_t total = E * static_cast<uint32_t>(a.H);
+  if (blockIdx.x >= total) return;  // uniform over the CTA
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_full[0][i], 1);
+      mbar_init(&sm.q_full[1][i], 1);
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.p_full[i][0], kBM);
       mbar_init(&sm.p_full[i][1], kBM);
       mbar_init(&sm.o_done[i], 1);
     }
-    mbar_init(&sm.q_empty, 1);
+    mbar_init(&sm.q_empty[0], 1);
+    mbar_init(&sm.q_empty[1], 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -228,22 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1)
    if (warp == kWarpLoad) {
     // ------------------------------------------------------------ loader
     if (lane == 0) {
-      uint32_t kv_it = 0, unit_it = 0, q0_loads = 0, q1_loads = 0, k_issued = 0, v_issued = 0;
+      uint32_t kv_it = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
-      for (long long u = blockIdx.x; u < total && ok; u += gridDim.x, ++unit_it) {
-        const Unit x = decode_unit(u, E, a.entries, a.cu_seqlens);
-        if (unit_it > 0 && !mbar_wait_bounded(&sm.q_empty, (unit_it - 1) & 1, abort_flag, dev_status)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&sm.q_full[0], kTileBytes);
-        tma_tile(sm.q[0], &tq, &sm.q_full[0], x.head, x.q0);
-        ++q0_loads;
-        if (x.has_q1) {
-          mbar_arrive_expect_tx(&sm.q_full[1], kTileBytes);
-          tma_tile(sm.q[1], &tq, &sm.q_full[1], x.head, x.q0 + kBM);
-          ++q1_loads;
-        }
+      for (UnitStream us(a.entries, E, total); us.valid() && ok;) {
+        const Unit x = us.take();
         for (int j = 0; j < x.nkv; ++j, ++kv_it) {
           const uint32_t st = kv_it % kStages, fill = kv_it / kStages;
           const int row0 = x.seg_start + j * kBN;
@@ -265,12 +288,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // Aborted: let the copies already issued land before the CTA exits.
-        if (q0_loads) mbar_wait_drain(&sm.q_full[0], (q0_loads - 1) & 1);
-        if (q1_loads) mbar_wait_drain(&sm.q_full[1], (q1_loads - 1) & 1);
         for (uint32_t f = (k_issued > kStages ? k_issued - kStages : 0); f < k_issued; ++f)
           mbar_wait_drain(&sm.k_full[f % kStages], (f / kStages) & 1);
         for (uint32_t f = (v_issued > kStages ? v_issued - kStages : 0); f < v_issued; ++f)
           mbar_wait_drain(&sm.v_full[f % kStages], (f / kStages) & 1);
+      }
+    }
+   } else if (warp == kWarpLoadQ) {
+    // ------------------------------------------------------------ Q loader
+    if (lane == 0) {
+      // per-buffer load counts (kept in scalars: a runtime-indexed array would go to local memory)
+      uint32_t unit_it = 0, q0a = 0, q0b = 0, q1a = 0, q1b = 0;
+      bool ok = true;
+      for (UnitStream us(a.entries, E, total); us.valid(); ++unit_it) {
+        const Unit x = us.take();
+        const uint32_t b = unit_it & 1, use = unit_it >> 1;
+        // buffer b is free once every QK of the unit that used it before has completed
+        if (use > 0 && !mbar_wait_bounded(&sm.q_empty[b], (use - 1) & 1, abort_flag, dev_status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&sm.q_full[b][0], kTileBytes);
+        tma_tile(sm.q[b][0], &tq, &sm.q_full[b][0], x.head, x.q0);
+        if (b) ++q0b; else ++q0a;
+        if (x.has_q1) {
+          mbar_arrive_expect_tx(&sm.q_full[b][1], kTileBytes);
+          tma_tile(sm.q[b][1], &tq, &sm.q_full[b][1], x.head, x.q0 + kBM);
+          if (b) ++q1b; else ++q1a;
+        }
+      }
+      if (!ok) {
+        // Aborted: let the copies already issued land before the CTA exits.
+        if (q0a) mbar_wait_drain(&sm.q_full[0][0], (q0a - 1) & 1);
+        if (q0b) mbar_wait_drain(&sm.q_full[1][0], (q0b - 1) & 1);
+        if (q1a) mbar_wait_drain(&sm.q_full[0][1], (q1a - 1) & 1);
+        if (q1b) mbar_wait_drain(&sm.q_full[1][1], (q1b - 1) & 1);
       }
     }
    } else if (warp == kWarpMma) {
@@ -278,16 +330,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = a.idesc_qk;
       const uint32_t idesc_pv = make_idesc_bf16(kBM, kDv, false, true, false);
-      const uint64_t dq0 = qk_desc(smem_u32(sm.q[0])), dq1 = qk_desc(smem_u32(sm.q[1]));
+      // Q buffer b, tile i starts (2 b + i) * kTileBytes after q[0][0]
+      const uint64_t dqbase = qk_desc(smem_u32(sm.q[0][0]));
       // stage s of the K (V) ring starts kTileBytes (kVTileBytes) after stage s-1
       const uint64_t dk0 = qk_desc(smem_u32(sm.k[0])), dv0 = pv_desc(smem_u32(sm.v[0]));
       auto dk = [&](uint32_t st) { return dk0 + static_cast<uint64_t>(st * (kTileBytes >> 4)); };
       auto dv = [&](uint32_t st) { return dv0 + static_cast<uint64_t>(st * (kVTileBytes >> 4)); };
-      uint32_t kv_it = 0, unit_it = 0, q1_it = 0, p_cnt0 = 0, p_cnt1 = 0;
-      for (long long u = blockIdx.x; u < total; u += gridDim.x, ++unit_it) {
-        const Unit x = decode_unit(u, E, a.entries, a.cu_seqlens);
-        if (!mbar_wait_bounded(&sm.q_full[0], unit_it & 1, abort_flag, dev_status)) break;
-        if (x.has_q1 && !mbar_wait_bounded(&sm.q_full[1], q1_it & 1, abort_flag, dev_status)) break;
+      uint32_t kv_it = 0, unit_it = 0, p_cnt0 = 0, p_cnt1 = 0;
+      uint32_t q1_it0 = 0, q1_it1 = 0;  // Q1 loads consumed per buffer
+      for (UnitStream us(a.entries, E, total); us.valid(); ++unit_it) {
+        const Unit x = us.take();
+        const uint32_t b = unit_it & 1;
+        const uint64_t dq0 = dqbase + static_cast<uint64_t>((2 * b) * (kTileBytes >> 4));
+        const uint64_t dq1 = dq0 + static_cast<uint64_t>(kTileBytes >> 4);
+        if (!mbar_wait_bounded(&sm.q_full[b][0], (unit_it >> 1) & 1, abort_flag, dev_status)) break;
+        if (x.has_q1 && !mbar_wait_bounded(&sm.q_full[b][1], (b ? q1_it1 : q1_it0) & 1, abort_flag, dev_status)) break;
         bool ok = true;
         {
           const uint32_t st = kv_it % kStages;
@@ -300,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&sm.s_full[1]);
           }
           mma_commit(&sm.k_empty[st]);
-          if (x.nkv == 1) mma_commit(&sm.q_empty);
+          if (x.nkv == 1) mma_commit(&sm.q_empty[b]);
         }
         for (int j = 0; j < x.nkv; ++j) {
           const uint32_t it = kv_it + j, st = it % kStages;
@@ -338,12 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&sm.v_empty[st]);
           if (more) {
             mma_commit(&sm.k_empty[st1]);
-            if (j + 2 == x.nkv) mma_commit(&sm.q_empty);
+            if (j + 2 == x.nkv) mma_commit(&sm.q_empty[b]);
           }
         }
         if (!ok) break;
         kv_it += x.nkv;
-        if (x.has_q1) ++q1_it;
+        if (x.has_q1) { if (b) ++q1_it1; else ++q1_it0; }
       }
       // All MMAs issued by this thread complete before TMEM is released.
       mma_commit(&sm.drain);
@@ -360,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + (wg ? kColO1 : kColO0);
     const float c = a.scale_log2;
     uint32_t s_cnt = 0, o_base = 0;
-    for (long long u = blockIdx.x; u < total; u += gridDim.x) {
-      const Unit x = decode_unit(u, E, a.entries, a.cu_seqlens);
+    for (UnitStream us(a.entries, E, total); us.valid();) {
+      const Unit x = us.take();
       if (wg == 1 && !x.has_q1) continue;
       const int row_tok = x.q0 + wg * kBM + r;
       float m = 0.f;
@@ -489,19 +546,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       reg_fence<kD + 1>(o);
       if (row_tok < x.seg_end) {
         const float inv_l = 1.0f / __uint_as_float(o[96]);
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) +
-                                              (static_cast<size_t>(row_tok) * a.H + x.head) * (kD * 2));
+        uint8_t* row = static_cast<uint8_t*>(a.out) +
+                       (static_cast<size_t>(row_tok) * a.H + x.head) * (kD * 2);
         const float2 il2 = make_float2(inv_l, inv_l);
+        uint32_t w[kD / 2];
 #pragma unroll
-        for (int i = 0; i < kD / 8; ++i) {
-          uint32_t w[4];
+        for (int i = 0; i < kD / 2; ++i) {
+          const float2 y = fmul2(make_float2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), il2);
+          w[i] = pack_bf16x2(y.x, y.y);
+        }
+        // a row is 192 contiguous bytes: six 32-byte stores (whole sectors) when the
+        // output is 32-byte aligned, else twelve 16-byte stores
+        if (a.out_align32) {
 #pragma unroll
-          for (int h2 = 0; h2 < 4; ++h2) {
-            const float2 y = fmul2(make_float2(__uint_as_float(o[8 * i + 2 * h2]),
-                                               __uint_as_float(o[8 * i + 2 * h2 + 1])), il2);
-            w[h2] = pack_bf16x2(y.x, y.y);
-          }
-          dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int i = 0; i < kD / 16; ++i) st_global_v8(row + 32 * i, w + 8 * i);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kD / 8; ++i)
+            reinterpret_cast<uint4*>(row)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
       o_base += x.nkv;

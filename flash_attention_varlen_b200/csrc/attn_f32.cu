@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(kThreads) attn_f32_kernel(const F32Args a) {
   for (long long u = blockIdx.x; u < total_units; u += gridDim.x) {
     const int e = static_cast<int>(u % E), h = static_cast<int>(u / E);
     const WorkEntry we = a.entries[e];
-    const int seg_start = a.cu_seqlens[we.seg], seg_end = a.cu_seqlens[we.seg + 1];
+    const int seg_start = we.seg_start, seg_end = we.seg_end;
     const int row = seg_start + we.qblock * kRows + r;
     const bool row_ok = row < seg_end;
 

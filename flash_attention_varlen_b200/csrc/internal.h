@@ -14,11 +14,15 @@ struct alignas(128) WorkHeader {
   int32_t pad[30];
 };
 
-// A work entry: one block of `block_rows` query rows of one segment.  The
-// kernels expand entry e and head h into unit u = h * E + e.
-struct WorkEntry {
+// A work entry: one block of `block_rows` query rows of one segment, stored
+// decoded (the segment's bounds included) so a kernel reads it with a single
+// 16-byte load it can issue a whole unit ahead.  The kernels expand entry e and
+// head h into unit u = h * E + e.
+struct alignas(16) WorkEntry {
   int32_t seg;
   int32_t qblock;
+  int32_t seg_start;  // cu_seqlens[seg]
+  int32_t seg_end;    // cu_seqlens[seg + 1]
 };
 
 // Entries that a call can produce at most: sum_s ceil(L_s / rows) <= T / rows + n.
@@ -48,6 +52,7 @@ struct Bf16Args {
   const WorkEntry* entries;
   int* dev_status;
   int32_t H;
+  int32_t out_align32;  // out is 32-byte aligned: rows go out as 256-bit stores
   float scale_log2;    // |scale| * log2(e)
   uint32_t idesc_qk;   // carries the sign of scale (negated A) for scale < 0
 };

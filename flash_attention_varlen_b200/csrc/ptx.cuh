@@ -57,6 +57,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed
+// sleeps until it does (or the hint, in ns, runs out) instead of spinning, so a
+// waiting warp leaves the issue slots of its SM sub-partition to the busy warps
+// beside it.
+constexpr uint32_t kSuspendHintNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity of `bar` has completed.  Gives up
 // (returns false) when another role of the CTA raised *abort, or after
 // kWaitTimeoutCycles, in which case it raises *abort and records a timeout in
@@ -66,8 +83,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((it & 7u) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > kWaitTimeoutCycles) {
         *abort_flag = 1;

@@ -88,15 +88,18 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
     // 2) entries per segment, exclusive scan, then write.  Thread t owns items 4t..4t+3.
-    int cnt[4], segs[4], local = 0;
+    int cnt[4], segs[4], starts[4], ends[4], local = 0;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int i = tid * 4 + r;
       cnt[r] = 0;
       segs[r] = 0;
+      starts[r] = ends[r] = 0;
       if (i < cn) {
         const int s = static_cast<int>(keys[i] & 0xFFFFFFFFull);
-        const int len = cu[s + 1] - cu[s];
+        starts[r] = cu[s];
+        ends[r] = cu[s + 1];
+        const int len = ends[r] - starts[r];
         segs[r] = s;
         cnt[r] = (len + block_rows - 1) / block_rows;
       }
@@ -115,7 +118,7 @@ __global__ void __launch_bounds__(kThreads)
     int off = base + warp_sums[warp] + incl - local;
 #pragma unroll
     for (int r = 0; r < 4; ++r)
-      for (int b = 0; b < cnt[r]; ++b) entries[off++] = WorkEntry{segs[r], b};
+      for (int b = 0; b < cnt[r]; ++b) entries[off++] = WorkEntry{segs[r], b, starts[r], ends[r]};
     base += chunk_total;
     __syncthreads();
   }

@@ -201,6 +201,7 @@ vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
     a.entries = entries;
     a.dev_status = &hdr->status;
     a.H = H;
+    a.out_align32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     const double log2e = 1.4426950408889634;
     a.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(scale)) * log2e);
     a.idesc_qk = vt::make_idesc_bf16(128, 128, false, false, scale < 0.0f);

@@ -26,7 +26,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB: header + 131056 entries
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB: header + 65528 entries
 constexpr int kMaxDevicesNoAlloc = 64;
 constexpr int kHeadDimNoAlloc = 96;
 
@@ -162,6 +162,7 @@ extern "C" vt_status vt_attn_fwd_noalloc(const void* q, const void* k, const voi
     a.entries = entries;
     a.dev_status = &hdr->status;
     a.H = H;
+    a.out_align32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     a.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(scale)) * 1.4426950408889634);
     a.idesc_qk = vt::make_idesc_bf16(128, 128, false, false, scale < 0.0f);
     const int grid = static_cast<int>(max_units < nd->num_sms ? max_units : nd->num_sms);

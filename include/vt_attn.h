@@ -89,9 +89,9 @@ vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
  * process exits) instead of a per-stream allocation.
  *
  * Limits and rules:
- *   - the work list must fit: 128 + 8 * (ceil(T / R) + num_segments) <= 1 MiB,
+ *   - the work list must fit: 128 + 16 * (ceil(T / R) + num_segments) <= 1 MiB,
  *     R = 256 for bf16, 64 for f32 (e.g. bf16 T = 16384 with 16 segments uses
- *     768 bytes); larger calls return VT_ERR_UNSUPPORTED and launch nothing;
+ *     1408 bytes); larger calls return VT_ERR_UNSUPPORTED and launch nothing;
  *   - the first call on a device looks up the array's device address for that
  *     device (make it with the device current, before capturing the stream into
  *     anything);

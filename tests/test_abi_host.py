@@ -73,9 +73,9 @@ def test_smem_contract(binding):
 
 
 def test_workspace_bytes(binding):
-    # header (128 B) + 8 B per entry, entries <= ceil(T / rows) + n
-    assert binding.vt_attn_workspace_bytes(16, 16384, binding.VT_DTYPE_BF16) == 128 + 8 * (64 + 16)
-    assert binding.vt_attn_workspace_bytes(1, 256, binding.VT_DTYPE_F32) == 128 + 8 * (4 + 1)
+    # header (128 B) + 16 B per entry, entries <= ceil(T / rows) + n
+    assert binding.vt_attn_workspace_bytes(16, 16384, binding.VT_DTYPE_BF16) == 128 + 16 * (64 + 16)
+    assert binding.vt_attn_workspace_bytes(1, 256, binding.VT_DTYPE_F32) == 128 + 16 * (4 + 1)
     assert binding.vt_attn_workspace_bytes(-1, 5, binding.VT_DTYPE_BF16) == 0
 
 

@@ -83,7 +83,7 @@ def test_noalloc_matches_vt_attn_fwd_on_two_calls_in_a_row():
 
 def test_noalloc_rejects_work_lists_beyond_its_array():
     from flash_attention_varlen_b200 import _binding as b
-    # 200000 one-token segments need 128 + 8 * (782 + 200000) bytes > 1 MiB: refused on the
+    # 200000 one-token segments need 128 + 16 * (782 + 200000) bytes > 1 MiB: refused on the
     # host before anything is launched (the pointers below are never dereferenced).
     T = n = 200000
     cu = np.zeros(4, np.int32)
