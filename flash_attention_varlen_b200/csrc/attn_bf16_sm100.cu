@@ -21,7 +21,9 @@
 //                        tensor core works on one tile while the other is in softmax.
 //   warps 0-3, 4-7     : softmax warpgroups for Q0 and Q1, one thread per row:
 //                        tcgen05.ld of the S row, row max (three-input max tree),
-//                        p = 2^(s*c - m) (packed f32x2 FMA, then MUFU ex2) with a
+//                        p = 2^(s*c - m) (packed f32x2 FMA, then MUFU ex2 for two
+//                        thirds of the pairs and a polynomial on the FMA pipe for
+//                        the rest) with a
 //                        deferred rescale (the running max m only moves when the
 //                        new tile max exceeds it by more than a threshold, so O in
 //                        TMEM is rarely touched), P packed to bf16 and written back
@@ -71,10 +73,12 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 // for a peaked softmax); 3 keeps a peaked (Q x 4) 1024-token row inside 1e-2 while
 // random N(0,1) rows almost never rescale.
 constexpr float kRescaleThreshold = 3.0f;
-// Every kPolyEvery-th pair of scores takes its exp2 on the FMA pipe (polynomial)
-// instead of the MUFU, which is otherwise the busiest unit (one exp2 per 384
-// tensor FLOPs at head width 96).  0 disables.
-constexpr int kPolyEvery = 0;
+// Every kPolyEvery-th pair of scores of a 64-key half (10 of 32 pairs for 3) takes
+// its exp2 on the FMA pipe (degree-3 minimax polynomial after Cody-Waite range
+// reduction, relative error 7.5e-5, far below the bf16 rounding of P) instead of the
+// MUFU, which is otherwise the busiest unit: one exp2 per 384 tensor FLOPs at head
+// width 96, and the MUFU issues 16 per clock per SM.  0 disables.
+constexpr int kPolyEvery = 3;
 
 static_assert(kBf16BlockRows == 2 * kBM, "a unit is two Q tiles");
 
@@ -197,6 +201,90 @@ __device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint
 #pragma unroll
   for (int c = 0; c < kD / 32; ++c)
     tma_load_3d(static_cast<uint8_t*>(dst) + c * kChunkBytes, map, bar, c * 32, head, row0);
+}
+
+// The MMA issuer (one thread).  It is kept out of line so that its loop is one compact
+// piece of code: the thread sleeps in mbarrier waits between short bursts of MMA
+// issue, and its wake-up latency is on the critical path of every key tile.
+__device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem, uint32_t E, uint32_t total,
+                                      volatile int* abort_flag, int* dev_status) {
+  const uint32_t idesc_qk = a.idesc_qk;
+  const uint32_t idesc_pv = make_idesc_bf16(kBM, kDv, false, true, false);
+  // Q buffer b, tile i starts (2 b + i) * kTileBytes after q[0][0]
+  const uint64_t dqbase = qk_desc(smem_u32(sm.q[0][0]));
+  // stage s of the K (V) ring starts kTileBytes (kVTileBytes) after stage s-1
+  const uint64_t dk0 = qk_desc(smem_u32(sm.k[0])), dv0 = pv_desc(smem_u32(sm.v[0]));
+  auto dk = [&](uint32_t st) { return dk0 + static_cast<uint64_t>(st * (kTileBytes >> 4)); };
+  auto dv = [&](uint32_t st) { return dv0 + static_cast<uint64_t>(st * (kVTileBytes >> 4)); };
+  uint32_t kv_it = 0, unit_it = 0, p_cnt0 = 0, p_cnt1 = 0;
+  uint32_t q1_it0 = 0, q1_it1 = 0;  // Q1 loads consumed per buffer
+  for (UnitStream us(a.entries, E, total); us.valid(); ++unit_it) {
+    const Unit x = us.take();
+    const uint32_t b = unit_it & 1;
+    const uint64_t dq0 = dqbase + static_cast<uint64_t>((2 * b) * (kTileBytes >> 4));
+    const uint64_t dq1 = dq0 + static_cast<uint64_t>(kTileBytes >> 4);
+    if (!mbar_wait_bounded(&sm.q_full[b][0], (unit_it >> 1) & 1, abort_flag, dev_status)) break;
+    if (x.has_q1 && !mbar_wait_bounded(&sm.q_full[b][1], (b ? q1_it1 : q1_it0) & 1, abort_flag, dev_status)) break;
+    bool ok = true;
+    {
+      const uint32_t st = kv_it % kStages;
+      if (!mbar_wait_bounded(&sm.k_full[st], (kv_it / kStages) & 1, abort_flag, dev_status)) break;
+      tc_fence_after();
+      issue_qk(tmem + kColS0, dq0, dk(st), idesc_qk);
+      mma_commit(&sm.s_full[0]);
+      if (x.has_q1) {
+        issue_qk(tmem + kColS1, dq1, dk(st), idesc_qk);
+        mma_commit(&sm.s_full[1]);
+      }
+      mma_commit(&sm.k_empty[st]);
+      if (x.nkv == 1) mma_commit(&sm.q_empty[b]);
+    }
+    for (int j = 0; j < x.nkv; ++j) {
+      const uint32_t it = kv_it + j, st = it % kStages;
+      const bool more = j + 1 < x.nkv;
+      const uint32_t st1 = (it + 1) % kStages;
+      if (!mbar_wait_bounded(&sm.v_full[st], (it / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
+      if (!mbar_wait_bounded(&sm.p_full[0][0], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
+      tc_fence_after();
+      issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 0, j > 0);
+      if (!mbar_wait_bounded(&sm.p_full[0][1], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
+      ++p_cnt0;
+      tc_fence_after();
+      issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 1, true);
+      mma_commit(&sm.o_done[0]);
+      if (more) {
+        if (!mbar_wait_bounded(&sm.k_full[st1], ((it + 1) / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
+        tc_fence_after();
+        issue_qk(tmem + kColS0, dq0, dk(st1), idesc_qk);
+        mma_commit(&sm.s_full[0]);
+      }
+      if (x.has_q1) {
+        if (!mbar_wait_bounded(&sm.p_full[1][0], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 0, j > 0);
+        if (!mbar_wait_bounded(&sm.p_full[1][1], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
+        ++p_cnt1;
+        tc_fence_after();
+        issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 1, true);
+        mma_commit(&sm.o_done[1]);
+        if (more) {
+          issue_qk(tmem + kColS1, dq1, dk(st1), idesc_qk);
+          mma_commit(&sm.s_full[1]);
+        }
+      }
+      mma_commit(&sm.v_empty[st]);
+      if (more) {
+        mma_commit(&sm.k_empty[st1]);
+        if (j + 2 == x.nkv) mma_commit(&sm.q_empty[b]);
+      }
+    }
+    if (!ok) break;
+    kv_it += x.nkv;
+    if (x.has_q1) { if (b) ++q1_it1; else ++q1_it0; }
+  }
+  // All MMAs issued by this thread complete before TMEM is released.
+  mma_commit(&sm.drain);
+  mbar_wait_drain(&sm.drain, 0);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -328,83 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
    } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_qk = a.idesc_qk;
-      const uint32_t idesc_pv = make_idesc_bf16(kBM, kDv, false, true, false);
-      // Q buffer b, tile i starts (2 b + i) * kTileBytes after q[0][0]
-      const uint64_t dqbase = qk_desc(smem_u32(sm.q[0][0]));
-      // stage s of the K (V) ring starts kTileBytes (kVTileBytes) after stage s-1
-      const uint64_t dk0 = qk_desc(smem_u32(sm.k[0])), dv0 = pv_desc(smem_u32(sm.v[0]));
-      auto dk = [&](uint32_t st) { return dk0 + static_cast<uint64_t>(st * (kTileBytes >> 4)); };
-      auto dv = [&](uint32_t st) { return dv0 + static_cast<uint64_t>(st * (kVTileBytes >> 4)); };
-      uint32_t kv_it = 0, unit_it = 0, p_cnt0 = 0, p_cnt1 = 0;
-      uint32_t q1_it0 = 0, q1_it1 = 0;  // Q1 loads consumed per buffer
-      for (UnitStream us(a.entries, E, total); us.valid(); ++unit_it) {
-        const Unit x = us.take();
-        const uint32_t b = unit_it & 1;
-        const uint64_t dq0 = dqbase + static_cast<uint64_t>((2 * b) * (kTileBytes >> 4));
-        const uint64_t dq1 = dq0 + static_cast<uint64_t>(kTileBytes >> 4);
-        if (!mbar_wait_bounded(&sm.q_full[b][0], (unit_it >> 1) & 1, abort_flag, dev_status)) break;
-        if (x.has_q1 && !mbar_wait_bounded(&sm.q_full[b][1], (b ? q1_it1 : q1_it0) & 1, abort_flag, dev_status)) break;
-        bool ok = true;
-        {
-          const uint32_t st = kv_it % kStages;
-          if (!mbar_wait_bounded(&sm.k_full[st], (kv_it / kStages) & 1, abort_flag, dev_status)) break;
-          tc_fence_after();
-          issue_qk(tmem + kColS0, dq0, dk(st), idesc_qk);
-          mma_commit(&sm.s_full[0]);
-          if (x.has_q1) {
-            issue_qk(tmem + kColS1, dq1, dk(st), idesc_qk);
-            mma_commit(&sm.s_full[1]);
-          }
-          mma_commit(&sm.k_empty[st]);
-          if (x.nkv == 1) mma_commit(&sm.q_empty[b]);
-        }
-        for (int j = 0; j < x.nkv; ++j) {
-          const uint32_t it = kv_it + j, st = it % kStages;
-          const bool more = j + 1 < x.nkv;
-          const uint32_t st1 = (it + 1) % kStages;
-          if (!mbar_wait_bounded(&sm.v_full[st], (it / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
-          if (!mbar_wait_bounded(&sm.p_full[0][0], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 0, j > 0);
-          if (!mbar_wait_bounded(&sm.p_full[0][1], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
-          ++p_cnt0;
-          tc_fence_after();
-          issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 1, true);
-          mma_commit(&sm.o_done[0]);
-          if (more) {
-            if (!mbar_wait_bounded(&sm.k_full[st1], ((it + 1) / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
-            tc_fence_after();
-            issue_qk(tmem + kColS0, dq0, dk(st1), idesc_qk);
-            mma_commit(&sm.s_full[0]);
-          }
-          if (x.has_q1) {
-            if (!mbar_wait_bounded(&sm.p_full[1][0], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 0, j > 0);
-            if (!mbar_wait_bounded(&sm.p_full[1][1], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
-            ++p_cnt1;
-            tc_fence_after();
-            issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 1, true);
-            mma_commit(&sm.o_done[1]);
-            if (more) {
-              issue_qk(tmem + kColS1, dq1, dk(st1), idesc_qk);
-              mma_commit(&sm.s_full[1]);
-            }
-          }
-          mma_commit(&sm.v_empty[st]);
-          if (more) {
-            mma_commit(&sm.k_empty[st1]);
-            if (j + 2 == x.nkv) mma_commit(&sm.q_empty[b]);
-          }
-        }
-        if (!ok) break;
-        kv_it += x.nkv;
-        if (x.has_q1) { if (b) ++q1_it1; else ++q1_it0; }
-      }
-      // All MMAs issued by this thread complete before TMEM is released.
-      mma_commit(&sm.drain);
-      mbar_wait_drain(&sm.drain, 0);
+      mma_role(sm, a, tmem, E, total, abort_flag, dev_status);
     }
    }
   } else {
@@ -432,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // pass 1, row max: the row in two 64-column halves, eight independent
         // three-input max chains
         float pm[8];
-#pragma unroll
+#pragma unroll 1  // one copy of the half body: a smaller hot loop for the instruction cache
         for (int half = 0; half < 2; ++half) {
           uint32_t su[kBN / 2];
           float* sf = reinterpret_cast<float*>(su);
@@ -499,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // pass 2: reload each half of S, exponentiate, store its P half (P half 0
         // overwrites S columns 0-31 only after that half has been read)
         const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
-#pragma unroll
+#pragma unroll 1  // one copy of the half body: a smaller hot loop for the instruction cache
         for (int half = 0; half < 2; ++half) {
           uint32_t su[kBN / 2];
           const float* sf = reinterpret_cast<const float*>(su);
@@ -510,9 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t p[kBN / 4];
 #pragma unroll
           for (int i2 = 0; i2 < kBN / 4; ++i2) {
-            const int i = half * (kBN / 4) + i2;
             const float2 t = ffma2(make_float2(sf[2 * i2], sf[2 * i2 + 1]), c2, nm2);
-            if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
+            if (kPolyEvery > 0 && i2 % kPolyEvery == kPolyEvery - 1) {
               const float2 e = exp2_poly2(t);  // FMA pipe: takes load off the MUFU
               p[i2] = pack_bf16x2(e.x, e.y);
             } else {
