@@ -31,6 +31,7 @@ EXPORTED = (
     "vt_attn_smem_bytes",
     "vt_attn_workspace_bytes",
     "vt_attn_last_device_status",
+    "vt_attn_selftest_wait_timeout",
     "vt_attn_status_string",
     "vt_attn_version",
 )
@@ -62,6 +63,8 @@ def _load():
     lib.vt_attn_workspace_bytes.restype = ctypes.c_size_t
     lib.vt_attn_last_device_status.argtypes = [P]
     lib.vt_attn_last_device_status.restype = ctypes.c_int
+    lib.vt_attn_selftest_wait_timeout.argtypes = [P, P, P, P, P, I32, I32, I32, I32, F, I32, P]
+    lib.vt_attn_selftest_wait_timeout.restype = ctypes.c_int
     lib.vt_attn_status_string.argtypes = [ctypes.c_int]
     lib.vt_attn_status_string.restype = ctypes.c_char_p
     lib.vt_attn_version.argtypes = []
@@ -102,6 +105,17 @@ def vt_attn_workspace_bytes(num_segments: int, total_tokens: int, dtype: int) ->
 
 def vt_attn_last_device_status(stream: int) -> int:
     return lib.vt_attn_last_device_status(stream)
+
+
+def vt_attn_selftest_wait_timeout(q: int, k: int, v: int, out: int, cu_seqlens: int,
+                                  num_segments: int, total_tokens: int, H: int, D: int,
+                                  scale: float, stall_cycles: int, stream: int) -> int:
+    """Failure-path self-test (bf16): the kernel's MMA thread waits on a barrier nothing
+    arrives on for stall_cycles cycles, then every role aborts; the device status of the
+    stream then reads VT_ERR_DEVICE_TIMEOUT.  Returns the launch status."""
+    return lib.vt_attn_selftest_wait_timeout(q, k, v, out, cu_seqlens, num_segments,
+                                             total_tokens, H, D, ctypes.c_float(scale),
+                                             stall_cycles, stream)
 
 
 def status_string(status: int) -> str:

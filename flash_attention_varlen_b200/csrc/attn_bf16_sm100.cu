@@ -96,6 +96,7 @@ struct Smem {
   uint64_t p_full[2][2];  // [Q tile][key half]: P columns 0-31 / 32-63 written
   uint64_t o_done[2];
   uint64_t drain;
+  uint64_t never;  // nothing arrives on it: the failure-path self-test waits here
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -208,6 +209,12 @@ __device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint
 // issue, and its wake-up latency is on the critical path of every key tile.
 __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem, uint32_t E, uint32_t total,
                                       volatile int* abort_flag, int* dev_status) {
+  if (a.stall_test_cycles > 0) {
+    // Failure-path self-test: this wait can never succeed, so it runs out after
+    // stall_test_cycles, raises the CTA's abort flag and records a timeout; every other
+    // role then leaves its loop exactly as after a real stall.  No MMA has been issued.
+    if (!mbar_wait_bounded(&sm.never, 0, abort_flag, dev_status, a.stall_test_cycles)) return;
+  }
   const uint32_t idesc_qk = a.idesc_qk;
   const uint32_t idesc_pv = make_idesc_bf16(kBM, kDv, false, true, false);
   // Q buffer b, tile i starts (2 b + i) * kTileBytes after q[0][0]
@@ -252,6 +259,10 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
       tc_fence_after();
       issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 1, true);
       mma_commit(&sm.o_done[0]);
+      // V_j is released as soon as its last PV has been issued (not behind the next QK):
+      // the loader refills the stage with V_{j+2}, and under full load a TMA tile takes
+      // ~3000 cycles to land, about one key tile of the ring's slack
+      if (!x.has_q1) mma_commit(&sm.v_empty[st]);
       if (more) {
         if (!mbar_wait_bounded(&sm.k_full[st1], ((it + 1) / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
         tc_fence_after();
@@ -267,12 +278,12 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
         tc_fence_after();
         issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 1, true);
         mma_commit(&sm.o_done[1]);
+        mma_commit(&sm.v_empty[st]);
         if (more) {
           issue_qk(tmem + kColS1, dq1, dk(st1), idesc_qk);
           mma_commit(&sm.s_full[1]);
         }
       }
-      mma_commit(&sm.v_empty[st]);
       if (more) {
         mma_commit(&sm.k_empty[st1]);
         if (j + 2 == x.nkv) mma_commit(&sm.q_empty[b]);
@@ -289,7 +300,7 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                     const __grid_constant__ CUtensorMap tv, const Bf16Args a) {
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ Bf16Args a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (raw & 1023u)) & 1023u));
@@ -317,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_empty[s], 1);
     }
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.never, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -374,8 +386,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++v_issued;
         }
       }
-      if (!ok) {
-        // Aborted: let the copies already issued land before the CTA exits.
+      {
+        // Every copy this thread issued has landed before the CTA exits.  Normally the MMA
+        // thread has already waited on each of them and these waits return at once; after
+        // an abort the last fills of the ring may still be in flight.  Only the last
+        // kStages fills per ring can be outstanding (each earlier one was waited on before
+        // its stage was refilled).
         for (uint32_t f = (k_issued > kStages ? k_issued - kStages : 0); f < k_issued; ++f)
           mbar_wait_drain(&sm.k_full[f % kStages], (f / kStages) & 1);
         for (uint32_t f = (v_issued > kStages ? v_issued - kStages : 0); f < v_issued; ++f)
@@ -387,15 +403,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // per-buffer load counts (kept in scalars: a runtime-indexed array would go to local memory)
       uint32_t unit_it = 0, q0a = 0, q0b = 0, q1a = 0, q1b = 0;
-      bool ok = true;
       for (UnitStream us(a.entries, E, total); us.valid(); ++unit_it) {
         const Unit x = us.take();
         const uint32_t b = unit_it & 1, use = unit_it >> 1;
         // buffer b is free once every QK of the unit that used it before has completed
-        if (use > 0 && !mbar_wait_bounded(&sm.q_empty[b], (use - 1) & 1, abort_flag, dev_status)) {
-          ok = false;
+        if (use > 0 && !mbar_wait_bounded(&sm.q_empty[b], (use - 1) & 1, abort_flag, dev_status))
           break;
-        }
         mbar_arrive_expect_tx(&sm.q_full[b][0], kTileBytes);
         tma_tile(sm.q[b][0], &tq, &sm.q_full[b][0], x.head, x.q0);
         if (b) ++q0b; else ++q0a;
@@ -405,8 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (b) ++q1b; else ++q1a;
         }
       }
-      if (!ok) {
-        // Aborted: let the copies already issued land before the CTA exits.
+      {
+        // Every Q copy issued has landed before the CTA exits (see the K/V loader).
         if (q0a) mbar_wait_drain(&sm.q_full[0][0], (q0a - 1) & 1);
         if (q0b) mbar_wait_drain(&sm.q_full[1][0], (q0b - 1) & 1);
         if (q1a) mbar_wait_drain(&sm.q_full[0][1], (q1a - 1) & 1);

@@ -55,6 +55,9 @@ struct Bf16Args {
   int32_t out_align32;  // out is 32-byte aligned: rows go out as 256-bit stores
   float scale_log2;    // |scale| * log2(e)
   uint32_t idesc_qk;   // carries the sign of scale (negated A) for scale < 0
+  // > 0 only in the failure-path self-test: the MMA thread first waits this many cycles
+  // on a barrier that never completes (see vt_attn_selftest_wait_timeout)
+  int32_t stall_test_cycles = 0;
 };
 size_t bf16_smem_bytes();
 cudaError_t prepare_attn_bf16();  // opt in to the kernel's dynamic shared memory (per device)

@@ -76,17 +76,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Wait until the phase with the given parity of `bar` has completed.  Gives up
 // (returns false) when another role of the CTA raised *abort, or after
-// kWaitTimeoutCycles, in which case it raises *abort and records a timeout in
+// `limit` cycles (kWaitTimeoutCycles unless given), in which case it raises *abort and records a timeout in
 // the device status word.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, int* dev_status) {
+                                                  volatile int* abort_flag, int* dev_status,
+                                                  long long limit = kWaitTimeoutCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_sleep(bar, parity)) return true;
     if ((it & 7u) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitTimeoutCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         atomicOr(dev_status, kDevStatusTimeout);
         return false;

@@ -142,9 +142,15 @@ size_t vt_attn_workspace_bytes(int32_t num_segments, int32_t total_tokens, vt_dt
   return vt::scratch_bytes_for(total_tokens, num_segments, block_rows_for(dtype));
 }
 
-vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
-                      const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
-                      int32_t H, int32_t D, float scale, vt_dtype dtype, void* stream_ptr) {
+}  // extern "C"
+
+namespace {
+
+// The forward; stall_test_cycles > 0 only for the failure-path self-test (bf16).
+vt_status fwd_impl(const void* q, const void* k, const void* v, void* out,
+                   const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                   int32_t H, int32_t D, float scale, vt_dtype dtype, void* stream_ptr,
+                   int32_t stall_test_cycles) {
   if (dtype != VT_DTYPE_BF16 && dtype != VT_DTYPE_F32) return VT_ERR_INVALID_ARG;
   if (H < 1 || D < 1 || num_segments < 0 || total_tokens < 0) return VT_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return VT_ERR_INVALID_ARG;
@@ -205,6 +211,7 @@ vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
     const double log2e = 1.4426950408889634;
     a.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(scale)) * log2e);
     a.idesc_qk = vt::make_idesc_bf16(128, 128, false, false, scale < 0.0f);
+    a.stall_test_cycles = stall_test_cycles;
     const int grid = static_cast<int>(max_units < di->num_sms ? max_units : di->num_sms);
     if (vt::launch_attn_bf16(tq, tk, tv, a, grid, stream) != cudaSuccess) return VT_ERR_CUDA;
   } else {
@@ -223,6 +230,27 @@ vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
     if (vt::launch_attn_f32(a, grid, stream) != cudaSuccess) return VT_ERR_CUDA;
   }
   return VT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                      const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                      int32_t H, int32_t D, float scale, vt_dtype dtype, void* stream_ptr) {
+  return fwd_impl(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D, scale, dtype,
+                  stream_ptr, 0);
+}
+
+vt_status vt_attn_selftest_wait_timeout(const void* q, const void* k, const void* v, void* out,
+                                        const int32_t* cu_seqlens, int32_t num_segments,
+                                        int32_t total_tokens, int32_t H, int32_t D, float scale,
+                                        int32_t stall_cycles, void* stream_ptr) {
+  if (stall_cycles < 1) return VT_ERR_INVALID_ARG;
+  if (num_segments < 1 || total_tokens < 1) return VT_ERR_INVALID_ARG;  // a kernel must run
+  return fwd_impl(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D, scale,
+                  VT_DTYPE_BF16, stream_ptr, stall_cycles);
 }
 
 vt_status vt_attn_last_device_status(void* stream_ptr) {

@@ -133,6 +133,30 @@ size_t vt_attn_workspace_bytes(int32_t num_segments, int32_t total_tokens, vt_dt
  */
 vt_status vt_attn_last_device_status(void* stream);
 
+/*
+ * Failure-path self-test of the bf16 kernel's bounded waits.  Every wait in the
+ * kernels is bounded.  In the vision-tower port commit of PR #279, a coverage
+ * check placed after its loop let a bad input hang instead of fail; this call
+ * exercises the bounded path on purpose, without a fault or a hang.
+ *
+ * Arguments are those of vt_attn_fwd for a valid bf16 problem (the same checks
+ * apply; at least one token), plus stall_cycles >= 1.  The call launches the
+ * bf16 forward, but in every CTA the MMA-issuing thread first waits on an
+ * mbarrier that nothing arrives on.  After stall_cycles SM clock cycles the wait
+ * gives up, raises the CTA's abort flag and records a timeout.  Every other role
+ * then leaves its loop, the TMA copies already issued are drained, and TMEM is
+ * released, as after a real stall.  No MMA is issued.
+ *
+ * Returns the launch status (VT_OK when launched).  A following
+ * vt_attn_last_device_status(stream) returns VT_ERR_DEVICE_TIMEOUT.  `out` is
+ * left unspecified.  The context stays usable, and the next vt_attn_fwd on the
+ * stream resets the device status.  Ownership is as for vt_attn_fwd.
+ */
+vt_status vt_attn_selftest_wait_timeout(const void* q, const void* k, const void* v, void* out,
+                                        const int32_t* cu_seqlens, int32_t num_segments,
+                                        int32_t total_tokens, int32_t H, int32_t D, float scale,
+                                        int32_t stall_cycles, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* vt_attn_status_string(vt_status status);
 

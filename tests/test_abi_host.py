@@ -117,3 +117,17 @@ def test_python_wrapper_refuses_cpu_tensors(binding):
     cu = torch.tensor([0, 4], dtype=torch.int32)
     with pytest.raises(ValueError):
         attn_fwd(q, q, q, cu)
+
+
+def test_selftest_wait_timeout_rejects_bad_arguments_on_host(binding):
+    f = binding.vt_attn_selftest_wait_timeout
+    cu, cup = _cu([0, 4])
+    P = 4096  # fake, never dereferenced: every call below fails a host check first
+    # the stall must be positive, and a kernel must actually run
+    assert f(P, P, P, P * 16, cup, 1, 4, 16, 96, 0.1, 0, 0) == binding.VT_ERR_INVALID_ARG
+    assert f(P, P, P, P * 16, cup, 1, 4, 16, 96, 0.1, -5, 0) == binding.VT_ERR_INVALID_ARG
+    assert f(0, 0, 0, 0, 0, 0, 0, 16, 96, 0.1, 1000, 0) == binding.VT_ERR_INVALID_ARG
+    # then the forward's own checks apply
+    assert f(P, P, P, P * 16, cup, 1, 4, 16, 64, 0.1, 1000, 0) == binding.VT_ERR_UNSUPPORTED
+    assert f(P, P, P, P * 16, 0, 1, 4, 16, 96, 0.1, 1000, 0) == binding.VT_ERR_NULL
+    assert f(P + 2, P, P, P * 16, cup, 1, 4, 16, 96, 0.1, 1000, 0) == binding.VT_ERR_INVALID_ARG
