@@ -7,6 +7,15 @@ computation is the library's CUDA kernels.
 
     out = attn_fwd(q, k, v, cu_seqlens)              # q/k/v: [T, 16, 96] bf16 or f32, cuda
     out = attn_fwd(q, k, v, cu_seqlens, scale=0.1)   # cu_seqlens: int32 [n+1] on the same device
+
+Window layers: ``window_partition`` builds, on the device, the order that makes every
+32 x 32-patch window of the images one contiguous segment, and ``permute_rows`` applies it
+(and its inverse) to [T, ...] tensors:
+
+    perm, cu = window_partition([(128, 128)], device=q.device)
+    qw = permute_rows(q, perm)                       # image order -> window order
+    ow = attn_fwd(qw, kw, vw, cu)
+    o = permute_rows(ow, perm, inverse=True)         # back to image order
 """
 from __future__ import annotations
 
@@ -17,7 +26,7 @@ from ._binding import (VT_DTYPE_BF16, VT_DTYPE_F32, VT_OK, VtAttnError, status_s
                        vt_attn_fwd, vt_attn_last_device_status, vt_attn_smem_bytes,
                        vt_attn_validate_seqlens_host, vt_attn_version, vt_attn_workspace_bytes)
 
-__all__ = ["attn_fwd", "attn_fwd_host", "check_device_status", "VtAttnError", "vt_attn_fwd",
+__all__ = ["attn_fwd", "attn_fwd_host", "window_partition", "permute_rows", "check_device_status", "VtAttnError", "vt_attn_fwd",
            "vt_attn_validate_seqlens_host", "vt_attn_smem_bytes", "vt_attn_workspace_bytes",
            "vt_attn_last_device_status", "status_string", "vt_attn_version"]
 
@@ -109,3 +118,52 @@ def attn_fwd_host(q_host, k_host, v_host, cu_host, out_host, scale: float | None
         attn_fwd(dq, dk, dv, dcu, scale=scale, out=do, stream=stream)
         out_host.copy_(do, non_blocking=True)
     return out_host
+
+
+def window_partition(grids, win: int = 32, device=None, stream=None):
+    """(perm, cu_seqlens) for images of patch grids ``grids`` = [(h, w), ...], on ``device``.
+
+    perm (int32 [T]): the packed image-order token at each position of the window order;
+    cu_seqlens (int32 [num_windows + 1]): the windows as segments of that order.
+    """
+    import ctypes
+    import torch
+    flat = [int(x) for hw in grids for x in hw]
+    if len(flat) != 2 * len(grids) or not grids:
+        raise ValueError("window_partition: grids must be a non-empty list of (h, w)")
+    g = (ctypes.c_int32 * len(flat))(*flat)
+    nw, nt = ctypes.c_int32(0), ctypes.c_int32(0)
+    rc = _binding.vt_window_count(ctypes.addressof(g), len(grids), win, ctypes.addressof(nw),
+                                  ctypes.addressof(nt))
+    if rc != VT_OK:
+        raise VtAttnError(rc, "vt_window_count")
+    device = torch.device("cuda") if device is None else torch.device(device)
+    perm = torch.empty(nt.value, dtype=torch.int32, device=device)
+    cu = torch.empty(nw.value + 1, dtype=torch.int32, device=device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    rc = _binding.vt_window_partition(ctypes.addressof(g), len(grids), win, perm.data_ptr(),
+                                      cu.data_ptr(), stream.cuda_stream)
+    if rc != VT_OK:
+        raise VtAttnError(rc, "vt_window_partition")
+    return perm, cu
+
+
+def permute_rows(x, perm, inverse: bool = False, out=None, stream=None):
+    """Rows of ``x`` ([T, ...] CUDA tensor) in the order ``perm`` (out[i] = x[perm[i]]), or,
+    with ``inverse``, put back (out[perm[i]] = x[i])."""
+    import torch
+    if not x.is_cuda or not perm.is_cuda or not x.is_contiguous():
+        raise ValueError("permute_rows: x and perm must be contiguous CUDA tensors")
+    if perm.dtype != torch.int32 or perm.dim() != 1 or perm.numel() != x.shape[0]:
+        raise ValueError("permute_rows: perm must be int32 [T] with T = x.shape[0]")
+    if out is None:
+        out = torch.empty_like(x)
+    row_bytes = x[0].numel() * x.element_size() if x.shape[0] else 16
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device)
+    rc = _binding.vt_permute_rows(x.data_ptr(), out.data_ptr(), perm.data_ptr(), x.shape[0],
+                                  row_bytes, 1 if inverse else 0, stream.cuda_stream)
+    if rc != VT_OK:
+        raise VtAttnError(rc, "vt_permute_rows")
+    return out

@@ -32,6 +32,9 @@ EXPORTED = (
     "vt_attn_workspace_bytes",
     "vt_attn_last_device_status",
     "vt_attn_selftest_wait_timeout",
+    "vt_window_count",
+    "vt_window_partition",
+    "vt_permute_rows",
     "vt_attn_status_string",
     "vt_attn_version",
 )
@@ -65,6 +68,12 @@ def _load():
     lib.vt_attn_last_device_status.restype = ctypes.c_int
     lib.vt_attn_selftest_wait_timeout.argtypes = [P, P, P, P, P, I32, I32, I32, I32, F, I32, P]
     lib.vt_attn_selftest_wait_timeout.restype = ctypes.c_int
+    lib.vt_window_count.argtypes = [P, I32, I32, P, P]
+    lib.vt_window_count.restype = ctypes.c_int
+    lib.vt_window_partition.argtypes = [P, I32, I32, P, P, P]
+    lib.vt_window_partition.restype = ctypes.c_int
+    lib.vt_permute_rows.argtypes = [P, P, P, I32, I32, I32, P]
+    lib.vt_permute_rows.restype = ctypes.c_int
     lib.vt_attn_status_string.argtypes = [ctypes.c_int]
     lib.vt_attn_status_string.restype = ctypes.c_char_p
     lib.vt_attn_version.argtypes = []
@@ -116,6 +125,24 @@ def vt_attn_selftest_wait_timeout(q: int, k: int, v: int, out: int, cu_seqlens: 
     return lib.vt_attn_selftest_wait_timeout(q, k, v, out, cu_seqlens, num_segments,
                                              total_tokens, H, D, ctypes.c_float(scale),
                                              stall_cycles, stream)
+
+
+def vt_window_count(grids_host: int, n_images: int, win: int, num_windows: int,
+                    total_tokens: int) -> int:
+    """Pure host: block and token counts of packed image grids (pointers as ints)."""
+    return lib.vt_window_count(grids_host, n_images, win, num_windows, total_tokens)
+
+
+def vt_window_partition(grids_host: int, n_images: int, win: int, perm: int, cu_seqlens: int,
+                        stream: int) -> int:
+    """Device window order of packed image grids: perm [T] and the blocks' cu_seqlens."""
+    return lib.vt_window_partition(grids_host, n_images, win, perm, cu_seqlens, stream)
+
+
+def vt_permute_rows(src: int, dst: int, index: int, num_rows: int, row_bytes: int, scatter: int,
+                    stream: int) -> int:
+    """dst[i] = src[index[i]] (scatter=0) or dst[index[i]] = src[i] (scatter=1), on the device."""
+    return lib.vt_permute_rows(src, dst, index, num_rows, row_bytes, scatter, stream)
 
 
 def status_string(status: int) -> str:

@@ -80,4 +80,18 @@ struct F32Args {
 size_t f32_smem_bytes();
 cudaError_t launch_attn_f32(const F32Args& args, int grid, cudaStream_t stream);
 
+// Window segmentation (window.cu).  Images are passed by value: at most kMaxWindowImages.
+constexpr int kMaxWindowImages = 64;
+struct WindowImages {
+  int32_t n, win;
+  int32_t h[kMaxWindowImages], w[kMaxWindowImages];
+  int64_t token_base[kMaxWindowImages + 1];   // packed image-order offset of each image
+  int64_t window_base[kMaxWindowImages + 1];  // index of each image's first block
+};
+cudaError_t launch_window_perm(const WindowImages& g, int32_t* perm, int32_t* cu, int num_sms,
+                               cudaStream_t stream);
+cudaError_t launch_permute_rows(const void* src, void* dst, const int32_t* idx, int32_t rows,
+                                int32_t row_bytes, int32_t scatter, int num_sms,
+                                cudaStream_t stream);
+
 }  // namespace vt

@@ -3,6 +3,7 @@
 // Host side only: argument validation, the per-(device, stream) scratch
 // buffer that holds the work list, TMA descriptors for the bf16 kernel, and
 // the two launches of a call (scheduling prepass, then the attention kernel).
+#include <climits>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -251,6 +252,88 @@ vt_status vt_attn_selftest_wait_timeout(const void* q, const void* k, const void
   if (num_segments < 1 || total_tokens < 1) return VT_ERR_INVALID_ARG;  // a kernel must run
   return fwd_impl(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D, scale,
                   VT_DTYPE_BF16, stream_ptr, stall_cycles);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Host-side description of the images for the window kernels; checks sizes and limits.
+vt_status window_images(const int32_t* grids, int32_t n_images, int32_t win, vt::WindowImages* g) {
+  if (!grids) return VT_ERR_NULL;
+  if (n_images < 1 || win < 1) return VT_ERR_INVALID_ARG;
+  if (n_images > vt::kMaxWindowImages) return VT_ERR_UNSUPPORTED;
+  g->n = n_images;
+  g->win = win;
+  g->token_base[0] = 0;
+  g->window_base[0] = 0;
+  for (int32_t i = 0; i < n_images; ++i) {
+    const int32_t h = grids[2 * i], w = grids[2 * i + 1];
+    if (h < 1 || w < 1) return VT_ERR_INVALID_ARG;
+    g->h[i] = h;
+    g->w[i] = w;
+    g->token_base[i + 1] = g->token_base[i] + static_cast<int64_t>(h) * w;
+    g->window_base[i + 1] = g->window_base[i] + static_cast<int64_t>((h + win - 1) / win) *
+                                                    ((w + win - 1) / win);
+    if (g->token_base[i + 1] > INT32_MAX) return VT_ERR_INVALID_ARG;
+  }
+  return VT_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+vt_status vt_window_count(const int32_t* grids, int32_t n_images, int32_t win,
+                          int32_t* num_windows, int32_t* total_tokens) {
+  vt::WindowImages g;
+  const vt_status st = window_images(grids, n_images, win, &g);
+  if (st != VT_OK) return st;
+  if (num_windows) *num_windows = static_cast<int32_t>(g.window_base[n_images]);
+  if (total_tokens) *total_tokens = static_cast<int32_t>(g.token_base[n_images]);
+  return VT_OK;
+}
+
+vt_status vt_window_partition(const int32_t* grids, int32_t n_images, int32_t win, int32_t* perm,
+                              int32_t* cu_seqlens, void* stream) {
+  vt::WindowImages g;
+  const vt_status st = window_images(grids, n_images, win, &g);
+  if (st != VT_OK) return st;
+  if (!perm || !cu_seqlens) return VT_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(perm) | reinterpret_cast<uintptr_t>(cu_seqlens)) & 3u)
+    return VT_ERR_INVALID_ARG;
+  const int nsm = sm_count();
+  if (nsm < 1) return VT_ERR_CUDA;
+  return vt::launch_window_perm(g, perm, cu_seqlens, nsm, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? VT_OK
+             : VT_ERR_CUDA;
+}
+
+vt_status vt_permute_rows(const void* src, void* dst, const int32_t* index, int32_t num_rows,
+                          int32_t row_bytes, int32_t scatter, void* stream) {
+  if (num_rows < 0 || row_bytes < 16 || (row_bytes & 15)) return VT_ERR_INVALID_ARG;
+  if (scatter != 0 && scatter != 1) return VT_ERR_INVALID_ARG;
+  if (num_rows == 0) return VT_OK;
+  if (!src || !dst || !index) return VT_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u)
+    return VT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(index) & 3u) return VT_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(num_rows) * row_bytes;
+  if (ranges_overlap(src, bytes, dst, bytes)) return VT_ERR_INVALID_ARG;
+  const int nsm = sm_count();
+  if (nsm < 1) return VT_ERR_CUDA;
+  return vt::launch_permute_rows(src, dst, index, num_rows, row_bytes, scatter, nsm,
+                                 static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? VT_OK
+             : VT_ERR_CUDA;
 }
 
 vt_status vt_attn_last_device_status(void* stream_ptr) {

@@ -157,6 +157,49 @@ vt_status vt_attn_selftest_wait_timeout(const void* q, const void* k, const void
                                         int32_t total_tokens, int32_t H, int32_t D, float scale,
                                         int32_t stall_cycles, void* stream);
 
+/*
+ * Window segmentation (the vision tower's window layers attend within 32 x 32-patch
+ * windows of each image: PR #279, "Two of the three labelled uncertainties are now
+ * resolved").  The tower puts its hidden states in window order once before its layers
+ * and back in image order once after them (PR #279, vision-tower port commit).  The
+ * calls below build that order on the device and apply it to [rows, ...] tensors.
+ *
+ * Order (the pages name the two orders without printing them; the plain row-major
+ * reading):
+ *   - images are packed one after another, each in row-major (y, x) patch order;
+ *   - an image's win x win blocks are walked row-major over its block grid, with smaller
+ *     blocks along the bottom and right edges when the grid is not a multiple of win;
+ *   - the tokens of a block are taken row-major inside it.
+ *
+ * grids: host array of n_images (h, w) pairs, 1 <= n_images <= 64, h, w >= 1, win >= 1,
+ * and the total token count must fit in int32 (else VT_ERR_INVALID_ARG /
+ * VT_ERR_UNSUPPORTED for more than 64 images).
+ *
+ * vt_window_count (pure host): the number of blocks and of tokens; either output
+ * pointer may be NULL.
+ */
+vt_status vt_window_count(const int32_t* grids, int32_t n_images, int32_t win,
+                          int32_t* num_windows, int32_t* total_tokens);
+
+/*
+ * Writes, on `stream`, perm[p] (device, int32 [total_tokens]) = the packed image-order
+ * token at position p of the window-ordered sequence, and cu_seqlens (device, int32
+ * [num_windows + 1]) delimiting the blocks in that sequence (the cu_seqlens a window
+ * layer passes to vt_attn_fwd).  Both buffers are the caller's, 4-byte aligned.
+ */
+vt_status vt_window_partition(const int32_t* grids, int32_t n_images, int32_t win,
+                              int32_t* perm, int32_t* cu_seqlens, void* stream);
+
+/*
+ * Row permutation on `stream`: scatter == 0 gathers dst[i] = src[index[i]] (image order
+ * to window order with index = perm); scatter == 1 scatters dst[index[i]] = src[i]
+ * (back).  Rows are row_bytes long (a multiple of 16, e.g. H * D * 2 for bf16
+ * [T, H, D]); src and dst are device pointers, 16-byte aligned, and must not overlap;
+ * index holds num_rows distinct row numbers in [0, num_rows).
+ */
+vt_status vt_permute_rows(const void* src, void* dst, const int32_t* index, int32_t num_rows,
+                          int32_t row_bytes, int32_t scatter, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* vt_attn_status_string(vt_status status);
 

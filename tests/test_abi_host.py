@@ -25,7 +25,7 @@ def binding():
 def _declared_functions():
     src = open(os.path.join(ROOT, "include", "vt_attn.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(vt_attn_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(vt_(?:attn|window|permute)_\w+)\s*\(", src)))
 
 
 def test_exports_every_declared_symbol(binding):
@@ -131,3 +131,27 @@ def test_selftest_wait_timeout_rejects_bad_arguments_on_host(binding):
     assert f(P, P, P, P * 16, cup, 1, 4, 16, 64, 0.1, 1000, 0) == binding.VT_ERR_UNSUPPORTED
     assert f(P, P, P, P * 16, 0, 1, 4, 16, 96, 0.1, 1000, 0) == binding.VT_ERR_NULL
     assert f(P + 2, P, P, P * 16, cup, 1, 4, 16, 96, 0.1, 1000, 0) == binding.VT_ERR_INVALID_ARG
+
+
+def test_window_count_on_host(binding):
+    import ctypes
+    def count(grids, win):
+        flat = [x for hw in grids for x in hw]
+        g = (ctypes.c_int32 * len(flat))(*flat)
+        nw, nt = ctypes.c_int32(-1), ctypes.c_int32(-1)
+        rc = binding.vt_window_count(ctypes.addressof(g), len(grids), win, ctypes.addressof(nw),
+                                     ctypes.addressof(nt))
+        return rc, nw.value, nt.value
+    assert count([(128, 128)], 32) == (binding.VT_OK, 16, 16384)
+    assert count([(40, 50)], 32) == (binding.VT_OK, 4, 2000)
+    assert count([(8, 8), (13, 29), (64, 33), (1, 1)], 8) == (binding.VT_OK, 1 + 8 + 40 + 1, 64 + 377 + 2112 + 1)
+    assert count([(0, 5)], 32)[0] == binding.VT_ERR_INVALID_ARG
+    assert count([(5, 5)], 0)[0] == binding.VT_ERR_INVALID_ARG
+    assert count([(1, 1)] * 65, 32)[0] == binding.VT_ERR_UNSUPPORTED
+    assert binding.vt_window_count(0, 1, 32, 0, 0) == binding.VT_ERR_NULL
+    # the device calls check their arguments on the host first
+    assert binding.vt_permute_rows(4096, 8192, 256, 4, 24, 0, 0) == binding.VT_ERR_INVALID_ARG  # row_bytes % 16
+    assert binding.vt_permute_rows(4096, 8192, 256, 4, 32, 2, 0) == binding.VT_ERR_INVALID_ARG  # scatter flag
+    assert binding.vt_permute_rows(4096, 4096 + 64, 256, 4, 32, 0, 0) == binding.VT_ERR_INVALID_ARG  # overlap
+    assert binding.vt_permute_rows(0, 8192, 256, 4, 32, 0, 0) == binding.VT_ERR_NULL
+    assert binding.vt_permute_rows(0, 0, 0, 0, 32, 0, 0) == binding.VT_OK  # nothing to move
