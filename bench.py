@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration timings of the smaller workloads")
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="steps of the host-buffer end-to-end measurement (default: min(steps, 3))")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -314,6 +316,10 @@ def run_ours(args):
     e2e = run_e2e(fa, torch, dev, pinned, cases, e2e_steps, step_flops, world,
                   dist if distributed else None)
 
+    # the other configurations of the workload, one layer each (informational): after the
+    # timed region, on this rank's GPU
+    configs = time_configs(fa, torch, dev) if not args.no_configs else None
+
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -354,6 +360,7 @@ def run_ours(args):
             "per_launch": "4*sum(L^2)*H*D FLOPs of the call / CUDA-event duration of the call, "
                           "averaged FLOP-weighted over the 50 calls of a step",
         },
+        "configs": configs,
         "gpu_launches": 2 * n_layers * args.steps,
         "e2e": e2e,
         "clocks": clock_info,
@@ -365,6 +372,46 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3):
+    """ms per call and TFLOP/s of each smaller configuration of the workload (one layer, the
+    inputs resident; calls back to back, so these small cases run partly out of L2)."""
+    cases = [workloads.tiny_case("bf16"), workloads.tiny_case("f32"), workloads.image448_case(),
+             workloads.image448_case(True), *workloads.image896_cases(), workloads.varlen8_case()]
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for c in cases:
+        q, k, v = c.inputs()
+        if c.dtype == "bf16":
+            to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+            code = fa.VT_DTYPE_BF16
+        else:
+            to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+            code = fa.VT_DTYPE_F32
+        dq, dk, dv = to(q), to(k), to(v)
+        do = torch.empty_like(dq)
+        cu = torch.from_numpy(c.cu_seqlens.copy()).to(dev)
+
+        def call():
+            rc = fa.vt_attn_fwd(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), do.data_ptr(),
+                                cu.data_ptr(), c.num_segments, c.T, c.H, c.D, SCALE, code,
+                                stream.cuda_stream)
+            if rc != 0:
+                raise fa.VtAttnError(rc, "vt_attn_fwd")
+        for _ in range(warmup):
+            call()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(calls):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        fa.check_device_status(stream)
+        ms = e0.elapsed_time(e1) / calls
+        out[c.name] = {"dtype": c.dtype, "segments": c.num_segments, "tokens": c.T,
+                       "ms": round(ms, 4), "tflops": round(c.flops() / (ms * 1e-3) / 1e12, 2)}
+    return out
 
 
 def run_e2e(fa, torch, dev, pinned, cases, steps, step_flops, world, dist):
