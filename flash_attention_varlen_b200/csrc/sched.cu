@@ -1,13 +1,13 @@
 // Scheduling prepass for the varlen attention kernels.
 //
 // The segments of one call (cu_seqlens, on the device) are cut into work
-// entries of `block_rows` query rows; the attention kernels then walk the
-// entries head-major (unit u -> head u / E, entry u % E) with a static stride
-// of gridDim.x.  Entries are ordered longest segment first, so the cheap units
-// come last and fill the tail wave (longest-processing-time-first list
-// scheduling).  Lengths are validated here, before any loop depends on them,
-// so a malformed cu_seqlens produces an empty work list and an error flag
-// instead of out-of-range reads.
+// entries of `block_rows` query rows, ordered longest segment first.  The bf16
+// kernel deals the units (entry, head) out in that order in a snake over its
+// CTAs, and the f32 kernel walks them head-major with a plain stride; either way
+// the cheap units come last and fill the tail (longest-processing-time-first list
+// scheduling).  Lengths are validated here, before any loop depends on them, so
+// a malformed cu_seqlens produces an empty work list and an error flag instead of
+// out-of-range reads.
 #include "internal.h"
 #include "ptx.cuh"
 
