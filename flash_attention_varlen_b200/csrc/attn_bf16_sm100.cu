@@ -108,21 +108,28 @@ struct Unit {
   bool has_q1;
 };
 
-// Walks this CTA's units.  Unit u is entry u / H of the work list for head u % H, so the
-// units come longest segment first (the prepass sorts the entries by segment length),
-// all heads of an entry together.  They are dealt to the CTAs in a snake: in round k, CTA
-// c takes unit k G + c when k is even and k G + G - 1 - c when k is odd (G CTAs).  With the
-// costs in decreasing order this pairs each round's expensive units with the next
-// round's cheap ones, a longest-processing-time-first approximation that needs no atomic
-// counter: on eight images of unequal size it balances the CTAs to within ~10-20% where a
-// plain stride left some with twice the mean.  Each unit is decoded from its 16-byte
-// entry, and the next unit's entry is loaded as soon as the current one is taken, so that
-// load's latency is hidden behind a whole unit of work instead of stalling every role at
-// each unit boundary.  The unit count stays below 2^31 (tokens x heads in device memory).
+// Walks this CTA's units (one per 256 query rows of one segment and head).  The units are
+// dealt to the CTAs in a snake: in round k, CTA c takes unit k G + c when k is even and
+// k G + G - 1 - c when k is odd (G CTAs).  Their order comes from the prepass:
+//  * segments of one length (a full layer; the windows of a window layer): head-major,
+//    unit u = entry u % E of head u / E, so the CTAs in flight share the K/V of a few
+//    heads in L2 (all heads at once would re-read K/V from HBM several times over);
+//  * segments of unequal length (a batch of images): entry-major, unit u = entry u / H
+//    of head u % H, so the units come longest segment first.  Dealt in a snake, each
+//    round's expensive units pair with the next round's cheap ones: a
+//    longest-processing-time-first approximation without an atomic counter (on eight
+//    images of unequal size it balances the CTAs to within ~10-20%, where a plain
+//    stride over head-major units left some with twice the mean).
+// Each unit is decoded from its 16-byte entry, and the next unit's entry is loaded as soon
+// as the current one is taken, so that load's latency is hidden behind a whole unit of
+// work instead of stalling every role at each unit boundary.  The unit count stays below
+// 2^31 (tokens x heads in device memory).
 class UnitStream {
  public:
-  __device__ __forceinline__ UnitStream(const WorkEntry* entries, uint32_t total, uint32_t H)
-      : entries_(reinterpret_cast<const int4*>(entries)), H_(H), total_(total) {
+  __device__ __forceinline__ UnitStream(const WorkEntry* entries, uint32_t E, uint32_t total,
+                                        uint32_t H, int order)
+      : entries_(reinterpret_cast<const int4*>(entries)), E_(E), H_(H), total_(total),
+        entry_major_(order != 0) {
     locate();
   }
   __device__ __forceinline__ bool valid() const { return u_ < total_; }
@@ -144,12 +151,19 @@ class UnitStream {
     const uint32_t c = blockIdx.x, G = gridDim.x;
     u_ = k_ * G + ((k_ & 1) ? G - 1 - c : c);
     if (u_ >= total_) return;
-    const uint32_t e = u_ / H_;
-    head_ = u_ - e * H_;
+    uint32_t e;
+    if (entry_major_) {
+      e = u_ / H_;
+      head_ = u_ - e * H_;
+    } else {
+      head_ = u_ / E_;
+      e = u_ - head_ * E_;
+    }
     cur_ = __ldg(entries_ + e);
   }
   const int4* entries_;
-  uint32_t H_, total_, k_ = 0, u_ = 0, head_ = 0;
+  uint32_t E_, H_, total_, k_ = 0, u_ = 0, head_ = 0;
+  bool entry_major_;
   int4 cur_ = make_int4(0, 0, 0, 0);
 };
 
@@ -215,7 +229,7 @@ __device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint
 // The MMA issuer (one thread).  It is kept out of line so that its loop is one compact
 // piece of code: the thread sleeps in mbarrier waits between short bursts of MMA
 // issue, and its wake-up latency is on the critical path of every key tile.
-__device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem, uint32_t total,
+__device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem, uint32_t E, uint32_t total,
                                       volatile int* abort_flag, int* dev_status) {
   if (a.stall_test_cycles > 0) {
     // Failure-path self-test: this wait can never succeed, so it runs out after
@@ -233,7 +247,7 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
   auto dv = [&](uint32_t st) { return dv0 + static_cast<uint64_t>(st * (kVTileBytes >> 4)); };
   uint32_t kv_it = 0, unit_it = 0, p_cnt0 = 0, p_cnt1 = 0;
   uint32_t q1_it0 = 0, q1_it1 = 0;  // Q1 loads consumed per buffer
-  for (UnitStream us(a.entries, total, a.H); us.valid(); ++unit_it) {
+  for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid(); ++unit_it) {
     const Unit x = us.take();
     const uint32_t b = unit_it & 1;
     const uint64_t dq0 = dqbase + static_cast<uint64_t>((2 * b) * (kTileBytes >> 4));
@@ -373,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kv_it = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
-      for (UnitStream us(a.entries, total, a.H); us.valid() && ok;) {
+      for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid() && ok;) {
         const Unit x = us.take();
         for (int j = 0; j < x.nkv; ++j, ++kv_it) {
           const uint32_t st = kv_it % kStages, fill = kv_it / kStages;
@@ -411,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // per-buffer load counts (kept in scalars: a runtime-indexed array would go to local memory)
       uint32_t unit_it = 0, q0a = 0, q0b = 0, q1a = 0, q1b = 0;
-      for (UnitStream us(a.entries, total, a.H); us.valid(); ++unit_it) {
+      for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid(); ++unit_it) {
         const Unit x = us.take();
         const uint32_t b = unit_it & 1, use = unit_it >> 1;
         // buffer b is free once every QK of the unit that used it before has completed
@@ -437,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
    } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      mma_role(sm, a, tmem, total, abort_flag, dev_status);
+      mma_role(sm, a, tmem, E, total, abort_flag, dev_status);
     }
    }
   } else {
@@ -450,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + (wg ? kColO1 : kColO0);
     const float c = a.scale_log2;
     uint32_t s_cnt = 0, o_base = 0;
-    for (UnitStream us(a.entries, total, a.H); us.valid();) {
+    for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid();) {
       const Unit x = us.take();
       if (wg == 1 && !x.has_q1) continue;
       const int row_tok = x.q0 + wg * kBM + r;

@@ -11,7 +11,12 @@ namespace vt {
 struct alignas(128) WorkHeader {
   int32_t status;       // kDevStatus* bit flags of the last call on this scratch
   int32_t num_entries;  // E: number of (segment, q-block) entries that follow
-  int32_t pad[30];
+  // Unit order of the bf16 kernel, set by the prepass: 0 = head-major (unit u = head u / E,
+  // entry u % E), for segments of one length: the CTAs in flight share few heads' K/V in
+  // L2; 1 = entry-major (entry u / H, head u % H), for segments of unequal length: the
+  // units come longest first, which the snake assignment needs to balance the CTAs
+  int32_t order;
+  int32_t pad[29];
 };
 
 // A work entry: one block of `block_rows` query rows of one segment, stored

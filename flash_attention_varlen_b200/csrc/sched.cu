@@ -2,10 +2,11 @@
 //
 // The segments of one call (cu_seqlens, on the device) are cut into work
 // entries of `block_rows` query rows, ordered longest segment first.  The bf16
-// kernel deals the units (entry, head) out in that order in a snake over its
-// CTAs, and the f32 kernel walks them head-major with a plain stride; either way
-// the cheap units come last and fill the tail (longest-processing-time-first list
-// scheduling).  Lengths are validated here, before any loop depends on them, so
+// kernel deals its units out in a snake over the CTAs, entry-major (longest
+// first) when the segments differ in length and head-major when they do not (the
+// header's order flag); the f32 kernel walks them head-major with a plain stride.
+// Either way the cheap units come last and fill the tail
+// (longest-processing-time-first list scheduling).  Lengths are validated here, before any loop depends on them, so
 // a malformed cu_seqlens produces an empty work list and an error flag instead of
 // out-of-range reads.
 #include "internal.h"
@@ -33,17 +34,30 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ unsigned long long keys[kSortMax];
   __shared__ int warp_sums[32];
   __shared__ int chunk_total;
+  __shared__ int len_min, len_max;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    len_min = 0x7FFFFFFF;
+    len_max = 0;
+  }
+  __syncthreads();
 
   // 1) validation: cu[0] == 0, cu[n] == T, non-decreasing.
   int bad = 0;
   if (tid == 0 && (cu[0] != 0 || cu[n] != T)) bad = 1;
-  for (int s = tid; s < n; s += kThreads)
-    if (cu[s + 1] < cu[s]) bad = 1;
+  for (int s = tid; s < n; s += kThreads) {
+    const int len = cu[s + 1] - cu[s];
+    if (len < 0) bad = 1;
+    if (len > 0) {  // the range of the non-empty lengths decides the unit order
+      atomicMin(&len_min, len);
+      atomicMax(&len_max, len);
+    }
+  }
   if (__syncthreads_or(bad)) {
     if (tid == 0) {
       hdr->status = kDevStatusBadSeqlens;
       hdr->num_entries = 0;
+      hdr->order = 0;
     }
     return;
   }
@@ -124,6 +138,7 @@ __global__ void __launch_bounds__(kThreads)
   }
   if (tid == 0) {
     hdr->num_entries = base;
+    hdr->order = (do_sort && len_min < len_max) ? 1 : 0;  // unequal lengths: longest first
     hdr->status = 0;
   }
 }
