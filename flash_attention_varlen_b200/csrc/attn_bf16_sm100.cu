@@ -23,11 +23,13 @@
 //                        tcgen05.ld of the S row, row max (three-input max tree),
 //                        p = 2^(s*c - m) (packed f32x2 FMA, then MUFU ex2 for two
 //                        thirds of the pairs and a polynomial on the FMA pipe for
-//                        the rest) with a
-//                        deferred rescale (the running max m only moves when the
-//                        new tile max exceeds it by more than a threshold, so O in
-//                        TMEM is rarely touched), P packed to bf16 and written back
-//                        over S in TMEM, then the epilogue O / l -> bf16 -> HBM.
+//                        the rest) with a deferred rescale (the running max m only
+//                        moves when the new tile max exceeds it by more than a
+//                        threshold, so O in TMEM is rarely touched), P packed to
+//                        bf16 and written back over S in TMEM, then the epilogue
+//                        O / l -> bf16 -> HBM.
+//
+// CTAs take their units in a longest-first snake order (see UnitStream).
 //
 // The row sum l is not accumulated by the softmax threads: each V stage carries
 // a fourth 32-column chunk whose first column is all ones, so column 96 of O
