@@ -134,6 +134,16 @@ def test_ragged_segments(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_more_segments_than_the_prepass_sorts(dtype):
+    # 5000 segments (the prepass sorts at most 4096: more keep their given order and
+    # are cut into entries chunk by chunk), lengths 0..40 drawn from the generator
+    lengths = workloads.uniform_int(7, 3, 5000, 0, 40)
+    cu = workloads.cu_from_lengths(lengths)
+    case = workloads.Case(f"many_segments_{dtype}", cu, seed=5, dtype=dtype)
+    _full_case(case)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("H", [1, 3])
 def test_other_head_counts(dtype, H):
     case = workloads.Case(f"H{H}_{dtype}", workloads.cu_from_lengths([300, 77, 129]), seed=4,
