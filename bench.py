@@ -12,8 +12,8 @@ Metric: attention TFLOP/s (FLOPs = 4 * sum(L^2) * H * D, block-diagonal work
 only) and ms per tower.  Prints ONE JSON line on rank 0.
 
 --impl reference times the CPU oracle (plain f64 C) on a bounded sample of the
-same workload; that is this build's reference arm (there is no other
-implementation of this path to run).
+same workload: the reference arm, since the source pages ship no runnable
+implementation of this path.
 """
 from __future__ import annotations
 

@@ -49,7 +49,7 @@ typedef enum {
   VT_OK = 0,
   VT_ERR_NULL = 1,           /* a required pointer is NULL */
   VT_ERR_INVALID_ARG = 2,    /* bad size, dtype, scale, alignment or aliasing */
-  VT_ERR_UNSUPPORTED = 3,    /* a valid request this build does not implement (D != 96) */
+  VT_ERR_UNSUPPORTED = 3,    /* a valid request the library does not implement (D != 96) */
   VT_ERR_BAD_SEQLENS = 4,    /* cu_seqlens not 0 = cu[0] <= ... <= cu[n] = total_tokens */
   VT_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed */
   VT_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up waiting on its own pipeline (bug guard) */
