@@ -122,3 +122,37 @@ def test_planted_mistakes_fail(mutant):
     perm, cu = mutant(grids, 32)
     with pytest.raises(AssertionError):
         _check(perm, cu, grids, 32)
+
+
+def _tiny_inputs(T, seed, H=2, D=8):
+    import workloads
+    return workloads.qkv(seed, T, H, D, "f32")
+
+
+def test_window_attention_single_window_is_plain_attention():
+    # a grid smaller than one window is a single segment: the permutation is the identity
+    import oracle
+    from oracle.window import window_attention
+    q, k, v = _tiny_inputs(5 * 7, 1)
+    got = window_attention(q, k, v, [(5, 7)], 0.3, win=8)
+    ref = oracle.attn_fwd(q, k, v, np.array([0, 35], np.int32), 0.3)
+    assert np.array_equal(got, ref)
+
+
+def test_window_attention_windows_are_independent():
+    # every window's output is attention over exactly that window's tokens, computed alone
+    import oracle
+    from oracle.window import window_attention
+    grids, win = [(6, 5), (3, 4)], 4
+    T = 6 * 5 + 3 * 4
+    q, k, v = _tiny_inputs(T, 2)
+    got = window_attention(q, k, v, grids, 0.5, win=win)
+    bases = [0, 30]
+    for img, (h, w) in enumerate(grids):
+        for by in range(0, h, win):
+            for bx in range(0, w, win):
+                toks = np.array([bases[img] + y * w + x for y in range(by, min(by + win, h))
+                                 for x in range(bx, min(bx + win, w))], np.int64)
+                cu = np.array([0, len(toks)], np.int32)
+                ref = oracle.attn_fwd(q[toks], k[toks], v[toks], cu, 0.5)
+                assert np.allclose(got[toks], ref, rtol=0, atol=1e-12)
