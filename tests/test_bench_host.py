@@ -1,0 +1,48 @@
+"""Host logic of bench.py that needs no GPU: the kernel-code fingerprint that decides
+whether the committed ncu DRAM counters still describe the kernel."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+SRC = """// header comment
+#include "x.h"
+/* block
+   comment */
+__global__ void k(int* a) {  // trailing comment
+  a[0] = 1;
+}
+"""
+
+
+def _fp(tmp_path, text):
+    p = tmp_path / "k.cu"
+    p.write_text(text)
+    old = bench.KERNEL_SRC
+    try:
+        bench.KERNEL_SRC = str(p)
+        return bench.kernel_sha()
+    finally:
+        bench.KERNEL_SRC = old
+
+
+def test_fingerprint_ignores_comments_and_whitespace(tmp_path):
+    base = _fp(tmp_path, SRC)
+    edited = SRC.replace("// header comment", "// a different header\n// over two lines")
+    edited = edited.replace("/* block\n   comment */", "/* reworded */")
+    edited = edited.replace("  a[0] = 1;", "      a[0]  =  1 ;")
+    assert _fp(tmp_path, edited) == base
+
+
+def test_fingerprint_follows_code(tmp_path):
+    base = _fp(tmp_path, SRC)
+    assert _fp(tmp_path, SRC.replace("a[0] = 1;", "a[0] = 2;")) != base
+    assert _fp(tmp_path, SRC.replace("int* a", "long* a")) != base
+
+
+def test_current_kernel_fingerprint_is_well_formed():
+    fp = bench.kernel_sha()
+    assert len(fp) == 16 and int(fp, 16) >= 0
