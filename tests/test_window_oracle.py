@@ -156,3 +156,12 @@ def test_window_attention_windows_are_independent():
                 cu = np.array([0, len(toks)], np.int32)
                 ref = oracle.attn_fwd(q[toks], k[toks], v[toks], cu, 0.5)
                 assert np.allclose(got[toks], ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("h,w", [(128, 128), (64, 64), (40, 50), (33, 97), (8, 8)])
+def test_matches_the_workload_window_lengths(h, w):
+    # the tower workloads build window-layer segments directly (workloads.window_lengths);
+    # they must be the segments of the window order
+    import workloads
+    _, cu = window_permutation([(h, w)], 32)
+    assert [int(x) for x in np.diff(cu)] == workloads.window_lengths(h, w)
