@@ -33,9 +33,16 @@ __global__ void __launch_bounds__(kThreads) attn_f32_kernel(const F32Args a) {
   const int H = a.H;
   const int E = a.hdr->num_entries;
   const long long total_units = static_cast<long long>(E) * H;
+  // the bf16 kernel's unit order: a snake over the CTAs, entry-major (longest segment
+  // first) when the segments differ in length and head-major when they do not
+  const bool entry_major = a.hdr->order != 0;
+  const long long G = gridDim.x, cta = blockIdx.x;
 
-  for (long long u = blockIdx.x; u < total_units; u += gridDim.x) {
-    const int e = static_cast<int>(u % E), h = static_cast<int>(u / E);
+  for (long long k = 0;; ++k) {
+    const long long u = k * G + ((k & 1) ? G - 1 - cta : cta);
+    if (u >= total_units) break;
+    const int e = static_cast<int>(entry_major ? u / H : u % E);
+    const int h = static_cast<int>(entry_major ? u % H : u / E);
     const WorkEntry we = a.entries[e];
     const int seg_start = we.seg_start, seg_end = we.seg_end;
     const int row = seg_start + we.qblock * kRows + r;

@@ -4,8 +4,8 @@
 // entries of `block_rows` query rows, ordered longest segment first.  The bf16
 // kernel deals its units out in a snake over the CTAs, entry-major (longest
 // first) when the segments differ in length and head-major when they do not (the
-// header's order flag); the f32 kernel walks them head-major with a plain stride.
-// Either way the cheap units come last and fill the tail
+// header's order flag), and the f32 kernel walks its units the same way.  The
+// cheap units come last and fill the tail
 // (longest-processing-time-first list scheduling).  Lengths are validated here, before any loop depends on them, so
 // a malformed cu_seqlens produces an empty work list and an error flag instead of
 // out-of-range reads.
