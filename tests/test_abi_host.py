@@ -155,3 +155,18 @@ def test_window_count_on_host(binding):
     assert binding.vt_permute_rows(4096, 4096 + 64, 256, 4, 32, 0, 0) == binding.VT_ERR_INVALID_ARG  # overlap
     assert binding.vt_permute_rows(0, 8192, 256, 4, 32, 0, 0) == binding.VT_ERR_NULL
     assert binding.vt_permute_rows(0, 0, 0, 0, 32, 0, 0) == binding.VT_OK  # nothing to move
+
+
+def test_window_wrappers_validate_on_host(binding):
+    import torch
+    import flash_attention_varlen_b200 as fa
+    with pytest.raises(ValueError):
+        fa.window_partition([])                      # no images
+    with pytest.raises(fa.VtAttnError):
+        fa.window_partition([(0, 4)])                # empty grid, refused by vt_window_count
+    with pytest.raises(fa.VtAttnError):
+        fa.window_partition([(4, 4)], win=0)
+    x = torch.zeros(4, 16, dtype=torch.float32)
+    perm = torch.arange(4, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        fa.permute_rows(x, perm)                     # CPU tensors: the library is GPU-only
