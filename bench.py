@@ -57,9 +57,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time budget of the oracle sample")
-    ap.add_argument("--single-layer", choices=["full", "window"], default=None,
-                    help="profiling aid: run only one tower layer (full = 1 x 16384 tok, "
-                         "window = 16 x 1024 tok) warmup + steps times and print its timing")
+    ap.add_argument("--single-layer", choices=["full", "window", "varlen8"], default=None,
+                    help="profiling aid: run only one layer (full = 1 x 16384 tok, window = "
+                         "16 x 1024 tok, varlen8 = eight images of unequal size) warmup + "
+                         "steps times and print its timing")
     return ap.parse_args(argv)
 
 
@@ -511,8 +512,10 @@ def run_single_layer(args):
     """One layer type of the tower, called warmup + steps times (for ncu captures)."""
     import torch
     import flash_attention_varlen_b200 as fa
-    layer = 3 if args.single_layer == "full" else 0
-    case = workloads.tower_layer_case(layer, GRID)
+    if args.single_layer == "varlen8":  # eight images of unequal size (the scheduler's case)
+        case = workloads.varlen8_case(0)
+    else:
+        case = workloads.tower_layer_case(3 if args.single_layer == "full" else 0, GRID)
     q, k, v = case.inputs()
     dev = torch.device("cuda", 0)
     to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
