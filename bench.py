@@ -412,7 +412,44 @@ def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3):
         ms = e0.elapsed_time(e1) / calls
         out[c.name] = {"dtype": c.dtype, "segments": c.num_segments, "tokens": c.T,
                        "ms": round(ms, 4), "tflops": round(c.flops() / (ms * 1e-3) / 1e12, 2)}
+    try:  # informational: must never cost the headline line
+        out["window_segmentation_128x128"] = time_window_segmentation(fa, torch, dev, calls)
+    except Exception as exc:  # noqa: BLE001
+        out["window_segmentation_128x128"] = {"error": str(exc)[:200]}
     return out
+
+
+def time_window_segmentation(fa, torch, dev, calls: int = 20):
+    """The tower image's window order built on the device, and one [16384, 16, 96] bf16
+    tensor put in that order (the tower does this once before its layers and once after)."""
+    stream = torch.cuda.current_stream(dev)
+    perm, cu = fa.window_partition([(GRID, GRID)], 32, device=dev)
+    x = torch.empty((GRID * GRID, workloads.HEADS, workloads.HEAD_DIM), dtype=torch.bfloat16,
+                    device=dev).normal_()
+    y = torch.empty_like(x)
+    for _ in range(3):
+        fa.window_partition([(GRID, GRID)], 32, device=dev)
+        fa.permute_rows(x, perm, out=y)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev[0].record(stream)
+    for _ in range(calls):
+        fa.window_partition([(GRID, GRID)], 32, device=dev)
+    ev[1].record(stream)
+    ev[2].record(stream)
+    for _ in range(calls):
+        fa.permute_rows(x, perm, out=y)
+    ev[3].record(stream)
+    torch.cuda.synchronize(dev)
+    part_ms = ev[0].elapsed_time(ev[1]) / calls
+    perm_ms = ev[2].elapsed_time(ev[3]) / calls
+    moved = 2 * x.numel() * x.element_size()  # read + write of every row
+    _, hbm_peak, _ = measured_peaks()
+    gbs = moved / (perm_ms * 1e-3) / 1e9
+    return {"partition_us": round(1e3 * part_ms, 2), "windows": int(cu.numel() - 1),
+            "permute_ms": round(perm_ms, 4), "permute_gbs": round(gbs, 1),
+            "permute_frac_of_hbm_peak": round(gbs / hbm_peak, 3) if hbm_peak else None,
+            "note": "partition includes its host-side checks and launch; permute moves "
+                    "2 x 50.3 MB per call"}
 
 
 def run_e2e(fa, torch, dev, pinned, cases, steps, step_flops, world, dist):
