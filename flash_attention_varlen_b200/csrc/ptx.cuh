@@ -328,11 +328,13 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 // 1.5 * 2^23 shift and f in [-1/2, 1/2]; 2^f ~ c0 + f (c1 + f (c2 + f c3)), the
 // degree-3 polynomial minimising the maximum relative error on [-1/2, 1/2]
 // (Remez exchange, fit_exp2_poly.py: 7.5e-5); 2^n enters by adding n to the
-// exponent field.  x is clamped at -127 (results below 2^-127 are not needed:
-// every row holds a 1 at its running max).
+// exponent field.  x is clamped at -126 (results below 2^-126 are not needed:
+// every row holds a 1 at its running max).  Not lower: with n = -127 a polynomial
+// value just below 1 (exponent field 126) would borrow into the sign bit and give a
+// NaN; from n >= -126 the smallest field is 0, a denormal of about the right size.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -127.0f);
-  x.y = fmaxf(x.y, -127.0f);
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
   const float2 shift = make_float2(12582912.0f, 12582912.0f);
   const float2 xi = fadd2(x, shift);
   const float2 n = fadd2(xi, make_float2(-12582912.0f, -12582912.0f));
