@@ -26,7 +26,9 @@ from ._binding import (VT_DTYPE_BF16, VT_DTYPE_F32, VT_OK, VtAttnError, status_s
                        vt_attn_fwd, vt_attn_last_device_status, vt_attn_smem_bytes,
                        vt_attn_validate_seqlens_host, vt_attn_version, vt_attn_workspace_bytes)
 
-__all__ = ["attn_fwd", "attn_fwd_host", "window_partition", "permute_rows", "check_device_status", "VtAttnError", "vt_attn_fwd",
+__all__ = ["attn_fwd", "attn_fwd_host", "window_partition", "permute_rows", "check_permute_rows",
+           "rope2d", "attn_fwd_rope2d",
+           "check_device_status", "VtAttnError", "vt_attn_fwd",
            "vt_attn_validate_seqlens_host", "vt_attn_smem_bytes", "vt_attn_workspace_bytes",
            "vt_attn_last_device_status", "status_string", "vt_attn_version"]
 
@@ -147,6 +149,81 @@ def window_partition(grids, win: int = 32, device=None, stream=None):
     if rc != VT_OK:
         raise VtAttnError(rc, "vt_window_partition")
     return perm, cu
+
+
+def attn_fwd_rope2d(q, k, v, cu_seqlens, pos, theta: float = 10000.0, scale: float | None = None,
+                    out=None, k_rot=None, stream=None):
+    """Block-diagonal attention over rope(Q), rope(K), V (bf16 [T, H, 96] CUDA tensors).
+
+    pos: int32 [T, 2] CUDA tensor of 1-based (pw, ph) per token.  Q is rotated inside the
+    kernel; K is rotated into ``k_rot`` (a new tensor unless given; ``k_rot=k`` rotates
+    in place).  Returns ``out``.
+    """
+    import torch
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("attn_fwd_rope2d: q, k, v must be bfloat16")
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("attn_fwd_rope2d: q, k, v must share a [T, H, D] shape")
+    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens", cu_seqlens), ("pos", pos)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"attn_fwd_rope2d: {name} must be a contiguous CUDA tensor")
+    if pos.dtype != torch.int32 or tuple(pos.shape) != (q.shape[0], 2):
+        raise ValueError("attn_fwd_rope2d: pos must be int32 [T, 2]")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+        raise TypeError("attn_fwd_rope2d: cu_seqlens must be a 1-D int32 tensor")
+    T, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = torch.empty_like(q) if out is None else out
+    k_rot = torch.empty_like(k) if k_rot is None else k_rot
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(q.device):
+        rc = _binding.vt_attn_fwd_rope2d(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                         cu_seqlens.data_ptr(), cu_seqlens.numel() - 1, T, H, D,
+                                         float(scale), pos.data_ptr(), float(theta),
+                                         k_rot.data_ptr(), handle)
+    if rc != VT_OK:
+        raise VtAttnError(rc, "vt_attn_fwd_rope2d")
+    return out
+
+
+def rope2d(x, pos, theta: float = 10000.0, out=None, stream=None):
+    """2D RoPE of a bf16 CUDA tensor x [T, H, 96] (width first, 1-based positions).
+
+    pos: int32 CUDA tensor [T, 2] of (pw, ph) = (column + 1, row + 1) per token.  Returns
+    ``out`` (a new tensor unless given; ``out=x`` rotates in place).
+    """
+    import torch
+    if not x.is_cuda or not pos.is_cuda or not x.is_contiguous() or not pos.is_contiguous():
+        raise ValueError("rope2d: x and pos must be contiguous CUDA tensors")
+    if x.dtype != torch.bfloat16 or x.dim() != 3:
+        raise TypeError("rope2d: x must be a bfloat16 [T, H, D] tensor")
+    if pos.dtype != torch.int32 or tuple(pos.shape) != (x.shape[0], 2):
+        raise ValueError("rope2d: pos must be int32 [T, 2]")
+    if out is None:
+        out = torch.empty_like(x)
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device)
+    T, H, D = x.shape
+    rc = _binding.vt_rope2d(x.data_ptr(), out.data_ptr(), pos.data_ptr(), T, H, D, float(theta),
+                            stream.cuda_stream)
+    if rc != VT_OK:
+        raise VtAttnError(rc, "vt_rope2d")
+    return out
+
+
+def check_permute_rows(stream=None, device=None):
+    """Synchronise the stream and raise if a ``permute_rows`` on this device skipped a row
+    whose index was outside [0, T) since the previous check (the flag is then cleared)."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    rc = _binding.vt_permute_rows_check(handle)
+    if rc != VT_OK:
+        raise VtAttnError(rc, "vt_permute_rows_check")
 
 
 def permute_rows(x, perm, inverse: bool = False, out=None, stream=None):

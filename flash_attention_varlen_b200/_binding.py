@@ -22,6 +22,7 @@ VT_ERR_UNSUPPORTED = 3
 VT_ERR_BAD_SEQLENS = 4
 VT_ERR_CUDA = 5
 VT_ERR_DEVICE_TIMEOUT = 6
+VT_ERR_BAD_INDEX = 7
 
 # every symbol include/vt_attn.h declares
 EXPORTED = (
@@ -35,6 +36,9 @@ EXPORTED = (
     "vt_window_count",
     "vt_window_partition",
     "vt_permute_rows",
+    "vt_permute_rows_check",
+    "vt_rope2d",
+    "vt_attn_fwd_rope2d",
     "vt_attn_status_string",
     "vt_attn_version",
 )
@@ -74,6 +78,12 @@ def _load():
     lib.vt_window_partition.restype = ctypes.c_int
     lib.vt_permute_rows.argtypes = [P, P, P, I32, I32, I32, P]
     lib.vt_permute_rows.restype = ctypes.c_int
+    lib.vt_attn_fwd_rope2d.argtypes = [P, P, P, P, P, I32, I32, I32, I32, F, P, F, P, P]
+    lib.vt_attn_fwd_rope2d.restype = ctypes.c_int
+    lib.vt_rope2d.argtypes = [P, P, P, I32, I32, I32, F, P]
+    lib.vt_rope2d.restype = ctypes.c_int
+    lib.vt_permute_rows_check.argtypes = [P]
+    lib.vt_permute_rows_check.restype = ctypes.c_int
     lib.vt_attn_status_string.argtypes = [ctypes.c_int]
     lib.vt_attn_status_string.restype = ctypes.c_char_p
     lib.vt_attn_version.argtypes = []
@@ -143,6 +153,26 @@ def vt_permute_rows(src: int, dst: int, index: int, num_rows: int, row_bytes: in
                     stream: int) -> int:
     """dst[i] = src[index[i]] (scatter=0) or dst[index[i]] = src[i] (scatter=1), on the device."""
     return lib.vt_permute_rows(src, dst, index, num_rows, row_bytes, scatter, stream)
+
+
+def vt_rope2d(x: int, out: int, pos: int, total_tokens: int, H: int, D: int, theta: float,
+              stream: int) -> int:
+    """out = 2D RoPE of x (bf16 [T, H, 96]; out may be x), pos int32 [T][2] 1-based (pw, ph)."""
+    return lib.vt_rope2d(x, out, pos, total_tokens, H, D, ctypes.c_float(theta), stream)
+
+
+def vt_attn_fwd_rope2d(q: int, k: int, v: int, out: int, cu_seqlens: int, num_segments: int,
+                       total_tokens: int, H: int, D: int, scale: float, pos: int, theta: float,
+                       k_rot: int, stream: int) -> int:
+    """Attention over rope(Q), rope(K) (bf16): Q rotated in the kernel, K into k_rot."""
+    return lib.vt_attn_fwd_rope2d(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D,
+                                  ctypes.c_float(scale), pos, ctypes.c_float(theta), k_rot, stream)
+
+
+def vt_permute_rows_check(stream: int) -> int:
+    """Synchronise `stream`; VT_ERR_BAD_INDEX if a permute on this device skipped an
+    out-of-range row index since the previous check (the flag is then cleared)."""
+    return lib.vt_permute_rows_check(stream)
 
 
 def status_string(status: int) -> str:

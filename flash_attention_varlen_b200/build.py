@@ -16,8 +16,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libvtattn.so")
 
-SOURCES = ["vt_attn.cu", "vt_attn_noalloc.cu", "sched.cu", "attn_bf16_sm100.cu", "attn_f32.cu", "window.cu"]
-HEADERS = ["ptx.cuh", "internal.h"]
+SOURCES = ["vt_attn.cu", "vt_attn_noalloc.cu", "sched.cu", "attn_bf16_sm100.cu", "attn_f32.cu",
+           "window.cu", "rope2d.cu"]
+HEADERS = ["ptx.cuh", "internal.h", "rope2d.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -9,7 +9,8 @@
 // One CTA (persistent, one per SM) works through units of 256 query rows of
 // one (segment, head): two 128-row Q tiles that share every K/V tile.
 //
-//   warps 8-11         : warp 8 loads K/V, warp 9 issues MMAs, warp 10 loads Q, 11 idle
+//   warps 8-11         : warp 8 loads K/V, warp 9 issues MMAs, warp 10 loads Q, warp 11
+//                        rotates Q by the 2D RoPE when the call asks for it
 //   warp 8  (K/V loader): TMA loads of K/V tiles into a 2-stage ring (64-byte
 //                        swizzled, 32-column chunks).
 //   warp 10 (Q loader) : TMA loads of Q0/Q1 into a double buffer, so the next
@@ -18,7 +19,11 @@
 //                          S_i = Q_i K_j^T     (SS, M128 N128 K96)  -> TMEM
 //                          O_i += P_i [V_j | 1] (TS, M128 N112 K128; P read from TMEM)
 //                        in the order S0 S1 | PV0 S0' | PV1 S1' | ... so that the
-//                        tensor core works on one tile while the other is in softmax.
+//                        tensor core works on one tile while the other is in softmax;
+//                        one flat stream over all units of the CTA, so a tile's first
+//                        S of the next unit follows its own last PV of this one.
+//   warp 11 (RoPE)     : only with a RoPE call: rotates each landed Q tile in shared
+//                        memory (2D RoPE, width first) before its QKs may read it.
 //   warps 0-3, 4-7     : softmax warpgroups for Q0 and Q1, one thread per row:
 //                        tcgen05.ld of the S row, row max (three-input max tree),
 //                        p = 2^(s*c - m) (packed f32x2 FMA, then MUFU ex2 for two
@@ -45,6 +50,7 @@
 // bounded and an abort flag lets all roles leave together.
 #include "internal.h"
 #include "ptx.cuh"
+#include "rope2d.cuh"
 
 namespace vt {
 namespace {
@@ -52,8 +58,9 @@ namespace {
 constexpr int kBM = 128;          // query rows per Q tile
 constexpr int kBN = 128;          // keys per K/V tile
 constexpr int kD = 96;            // head width
-constexpr int kStages = 2;        // K/V ring depth
-constexpr int kQBufs = 2;         // Q is double-buffered: the next unit's Q lands during this one
+constexpr int kKStages = 2;  // K ring depth
+constexpr int kVStages = 2;  // V ring depth
+constexpr int kQBufs = 2;    // Q is double-buffered: the next unit's Q lands during this one
 constexpr int kDv = kD + 16;               // PV N: 96 value columns + ones column (+15 zero)
 constexpr int kTileBytes = kBM * kD * 2;   // 24576: a 128-row Q or K tile
 constexpr int kChunkBytes = 128 * 64;      // 8192: 128 rows x 32 bf16
@@ -67,6 +74,7 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "regi
 constexpr int kWarpLoad = 8;       // K/V loader
 constexpr int kWarpMma = 9;
 constexpr int kWarpLoadQ = 10;     // Q loader (runs up to one unit ahead)
+constexpr int kWarpRope = 11;      // 2D RoPE of the Q tiles (when enabled)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 // The running max only moves when a tile's max exceeds it by more than this (log2
@@ -81,21 +89,30 @@ constexpr float kRescaleThreshold = 3.0f;
 // MUFU, which is otherwise the busiest unit: one exp2 per 384 tensor FLOPs at head
 // width 96, and the MUFU issues 16 per clock per SM.  0 disables.
 constexpr int kPolyEvery = 3;
+// P is handed to the PV product in two key halves: the product of the first 64 keys
+// runs while the softmax still exponentiates the other 64.
+constexpr int kPChunks = 2;
 
 static_assert(kBf16BlockRows == 2 * kBM, "a unit is two Q tiles");
+// waits of the MMA thread
+__device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         int* dev_status) {
+  return mbar_wait_bounded(bar, parity, abort_flag, dev_status);
+}
 
 struct Smem {
   uint8_t q[kQBufs][2][kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kVTileBytes];
+  uint8_t k[kKStages][kTileBytes];
+  uint8_t v[kVStages][kVTileBytes];
   uint64_t q_full[kQBufs][2];
   uint64_t q_empty[kQBufs];
-  uint64_t k_full[kStages];
-  uint64_t k_empty[kStages];
-  uint64_t v_full[kStages];
-  uint64_t v_empty[kStages];
+  uint64_t q_ready[kQBufs][2];  // RoPE prologue: the landed Q tile has been rotated
+  uint64_t k_full[kKStages];
+  uint64_t k_empty[kKStages];
+  uint64_t v_full[kVStages];
+  uint64_t v_empty[kVStages];
   uint64_t s_full[2];
-  uint64_t p_full[2][2];  // [Q tile][key half]: P columns 0-31 / 32-63 written
+  uint64_t p_full[2][kPChunks];  // [Q tile][key chunk]: that chunk's P columns written
   uint64_t o_done[2];
   uint64_t drain;
   uint64_t never;  // nothing arrives on it: the failure-path self-test waits here
@@ -201,16 +218,30 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint6
 __device__ __forceinline__ uint64_t pv_desc(uint32_t saddr) {
   return make_smem_desc(saddr, kChunkBytes, 512, kSwizzle64B);
 }
-// One half of the K loop (keys 64*half .. +63), so the product can start on the
-// first 64 keys while the softmax still computes the other 64.
-__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
-                                              uint32_t idesc, int half, bool accumulate) {
+// One key chunk of the K loop (keys chunk * 128 / kPChunks onwards), so the product can
+// start on the first keys while the softmax still computes the others.
+__device__ __forceinline__ void issue_pv_chunk(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
+                                               uint32_t idesc, int chunk, bool accumulate) {
+  constexpr int kSteps = (kBN / 16) / kPChunks;  // K16 steps per chunk
 #pragma unroll
-  for (int k4 = 0; k4 < kBN / 32; ++k4) {
-    const int kk = half * (kBN / 32) + k4;
+  for (int s = 0; s < kSteps; ++s) {
+    const int kk = chunk * kSteps + s;
     mma_ts(d_tmem, p_tmem + kk * 8, v_desc + static_cast<uint64_t>((kk * 1024) >> 4), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
   }
+}
+
+// O_i += P_i [V | 1] for one key tile, chunk by chunk as the softmax releases P.
+__device__ __forceinline__ bool issue_pv(Smem& sm, int tile, uint32_t d_tmem, uint32_t p_tmem,
+                                         uint64_t v_desc, uint32_t idesc, uint32_t parity,
+                                         bool accumulate, volatile int* abort_flag, int* dev_status) {
+#pragma unroll
+  for (int c = 0; c < kPChunks; ++c) {
+    if (!mma_wait(&sm.p_full[tile][c], parity, abort_flag, dev_status)) return false;
+    tc_fence_after();
+    issue_pv_chunk(d_tmem, p_tmem, v_desc, idesc, c, accumulate);
+  }
+  return true;
 }
 
 // Every lane waits; the outcome is made warp-uniform because the tcgen05.ld/st
@@ -226,6 +257,34 @@ __device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint
 #pragma unroll
   for (int c = 0; c < kD / 32; ++c)
     tma_load_3d(static_cast<uint8_t*>(dst) + c * kChunkBytes, map, bar, c * 32, head, row0);
+}
+
+// 2D RoPE of one landed 128-row Q tile in shared memory (three 32-column chunks, 64-byte
+// swizzle: 16-byte unit u of row r sits at unit u ^ ((r >> 1) & 3)), by one warp: lane l
+// rotates rows l, l + 32, l + 64, l + 96, each as six (group, group + 6) pairs of 16-byte
+// groups (columns 8g .. 8g + 7 with 48 + 8g .. 48 + 8g + 7).  Rows past the segment end
+// are left as they are: they are computed but never stored.
+__device__ __forceinline__ void rope_q_tile(uint8_t* tile, const int32_t* pos, int row_tok0,
+                                            int seg_end, const float* freq, int lane) {
+#pragma unroll 1
+  for (int k = 0; k < 4; ++k) {
+    const int r = lane + 32 * k;
+    const int tok = row_tok0 + r;
+    if (tok >= seg_end) continue;
+    const int2 p = __ldg(reinterpret_cast<const int2*>(pos) + tok);
+    const float pw = static_cast<float>(p.x), ph = static_cast<float>(p.y);
+    const uint32_t sw = (r >> 1) & 3;
+#pragma unroll 1
+    for (int g = 0; g < 6; ++g) {
+      const int g2 = g + 6;
+      uint4* plo = reinterpret_cast<uint4*>(tile + (g >> 2) * kChunkBytes + r * 64 + (((g & 3) ^ sw) << 4));
+      uint4* phi = reinterpret_cast<uint4*>(tile + (g2 >> 2) * kChunkBytes + r * 64 + (((g2 & 3) ^ sw) << 4));
+      uint4 lo = *plo, hi = *phi;
+      rope_rotate_group(lo, hi, g, pw, ph, freq);
+      *plo = lo;
+      *phi = hi;
+    }
+  }
 }
 
 // The MMA issuer (one thread).  It is kept out of line so that its loop is one compact
@@ -245,77 +304,100 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
   const uint64_t dqbase = qk_desc(smem_u32(sm.q[0][0]));
   // stage s of the K (V) ring starts kTileBytes (kVTileBytes) after stage s-1
   const uint64_t dk0 = qk_desc(smem_u32(sm.k[0])), dv0 = pv_desc(smem_u32(sm.v[0]));
-  auto dk = [&](uint32_t st) { return dk0 + static_cast<uint64_t>(st * (kTileBytes >> 4)); };
+  auto dk = [&](uint32_t st) { return dk0 + static_cast<uint64_t>(st * (kTileBytes >> 4)); };  // K stage
   auto dv = [&](uint32_t st) { return dv0 + static_cast<uint64_t>(st * (kVTileBytes >> 4)); };
+  auto dq = [&](uint32_t b, int tile) {
+    return dqbase + static_cast<uint64_t>((2 * b + tile) * (kTileBytes >> 4));
+  };
   uint32_t kv_it = 0, unit_it = 0, p_cnt0 = 0, p_cnt1 = 0;
   uint32_t q1_it0 = 0, q1_it1 = 0;  // Q1 loads consumed per buffer
-  for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid(); ++unit_it) {
-    const Unit x = us.take();
-    const uint32_t b = unit_it & 1;
-    const uint64_t dq0 = dqbase + static_cast<uint64_t>((2 * b) * (kTileBytes >> 4));
-    const uint64_t dq1 = dq0 + static_cast<uint64_t>(kTileBytes >> 4);
-    if (!mbar_wait_bounded(&sm.q_full[b][0], (unit_it >> 1) & 1, abort_flag, dev_status)) break;
-    if (x.has_q1 && !mbar_wait_bounded(&sm.q_full[b][1], (b ? q1_it1 : q1_it0) & 1, abort_flag, dev_status)) break;
-    bool ok = true;
-    {
-      const uint32_t st = kv_it % kStages;
-      if (!mbar_wait_bounded(&sm.k_full[st], (kv_it / kStages) & 1, abort_flag, dev_status)) break;
+  // Q of unit number n (buffer n % kQBufs) has landed
+  // (with the RoPE prologue: has been rotated in shared memory)
+  uint64_t(*qbar)[2] = a.rope_pos != nullptr ? sm.q_ready : sm.q_full;
+  auto wait_q = [&](const Unit& u, uint32_t n) {
+    const uint32_t b = n % kQBufs;
+    if (!mma_wait(&qbar[b][0], (n / kQBufs) & 1, abort_flag, dev_status)) return false;
+    if (u.has_q1 && !mma_wait(&qbar[b][1], (b ? q1_it1 : q1_it0) & 1, abort_flag, dev_status))
+      return false;
+    return true;
+  };
+  // The issue order is one flat stream over all key tiles of all units of this CTA:
+  //   PV0(j) | QK0(j+1) | PV1(j) | QK1(j+1)
+  // where tile j+1 after a unit's last tile is the next unit's first.  So a Q tile's next S
+  // is computed right after its own last PV of a unit (during that tile's epilogue), not
+  // behind the other tile's last PV.  The K/V ring runs on across units as the loader fills it.
+  UnitStream us(a.entries, E, total, a.H, a.hdr->order);
+  bool ok = us.valid();
+  Unit x;
+  if (ok) {
+    x = us.take();
+    ok = wait_q(x, 0);
+  }
+  if (ok) {
+    const uint32_t st = 0, b = 0;
+    ok = mma_wait(&sm.k_full[st], 0, abort_flag, dev_status);
+    if (ok) {
       tc_fence_after();
-      issue_qk(tmem + kColS0, dq0, dk(st), idesc_qk);
+      issue_qk(tmem + kColS0, dq(b, 0), dk(st), idesc_qk);
       mma_commit(&sm.s_full[0]);
       if (x.has_q1) {
-        issue_qk(tmem + kColS1, dq1, dk(st), idesc_qk);
+        issue_qk(tmem + kColS1, dq(b, 1), dk(st), idesc_qk);
         mma_commit(&sm.s_full[1]);
       }
       mma_commit(&sm.k_empty[st]);
       if (x.nkv == 1) mma_commit(&sm.q_empty[b]);
     }
+  }
+  while (ok) {
+    // S(x, 0) has been issued for both tiles
+    const uint32_t b = unit_it % kQBufs, b2 = (unit_it + 1) % kQBufs;
+    const bool has_next = us.valid();
+    Unit y = x;
+    if (has_next) y = us.take();
     for (int j = 0; j < x.nkv; ++j) {
-      const uint32_t it = kv_it + j, st = it % kStages;
-      const bool more = j + 1 < x.nkv;
-      const uint32_t st1 = (it + 1) % kStages;
-      if (!mbar_wait_bounded(&sm.v_full[st], (it / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
-      if (!mbar_wait_bounded(&sm.p_full[0][0], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
-      tc_fence_after();
-      issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 0, j > 0);
-      if (!mbar_wait_bounded(&sm.p_full[0][1], p_cnt0 & 1, abort_flag, dev_status)) { ok = false; break; }
+      const uint32_t it = kv_it + j, st = it % kVStages;
+      const bool last = j + 1 == x.nkv;
+      const bool more = !last || has_next;  // a QK follows: this unit's next tile or y's first
+      const uint32_t st1 = (it + 1) % kKStages;
+      const uint32_t nb = last ? b2 : b;                  // Q buffer of that QK
+      const bool next_q1 = last ? y.has_q1 : x.has_q1;    // ... and whether it has tile 1
+      if (!mma_wait(&sm.v_full[st], (it / kVStages) & 1, abort_flag, dev_status)) { ok = false; break; }
+      if (!issue_pv(sm, 0, tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, p_cnt0 & 1, j > 0,
+                    abort_flag, dev_status)) { ok = false; break; }
       ++p_cnt0;
-      tc_fence_after();
-      issue_pv_half(tmem + kColO0, tmem + kColS0, dv(st), idesc_pv, 1, true);
       mma_commit(&sm.o_done[0]);
-      // V_j is released as soon as its last PV has been issued (not behind the next QK):
-      // the loader refills the stage with V_{j+2}, and under full load a TMA tile takes
-      // ~3000 cycles to land, about one key tile of the ring's slack
+      // V_j is released as soon as its last PV has been issued (not behind the next QK)
       if (!x.has_q1) mma_commit(&sm.v_empty[st]);
       if (more) {
-        if (!mbar_wait_bounded(&sm.k_full[st1], ((it + 1) / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
+        if (last && !wait_q(y, unit_it + 1)) { ok = false; break; }
+        if (!mma_wait(&sm.k_full[st1], ((it + 1) / kKStages) & 1, abort_flag, dev_status)) { ok = false; break; }
         tc_fence_after();
-        issue_qk(tmem + kColS0, dq0, dk(st1), idesc_qk);
+        issue_qk(tmem + kColS0, dq(nb, 0), dk(st1), idesc_qk);
         mma_commit(&sm.s_full[0]);
       }
       if (x.has_q1) {
-        if (!mbar_wait_bounded(&sm.p_full[1][0], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 0, j > 0);
-        if (!mbar_wait_bounded(&sm.p_full[1][1], p_cnt1 & 1, abort_flag, dev_status)) { ok = false; break; }
+        if (!issue_pv(sm, 1, tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, p_cnt1 & 1, j > 0,
+                      abort_flag, dev_status)) { ok = false; break; }
         ++p_cnt1;
-        tc_fence_after();
-        issue_pv_half(tmem + kColO1, tmem + kColS1, dv(st), idesc_pv, 1, true);
         mma_commit(&sm.o_done[1]);
         mma_commit(&sm.v_empty[st]);
-        if (more) {
-          issue_qk(tmem + kColS1, dq1, dk(st1), idesc_qk);
-          mma_commit(&sm.s_full[1]);
-        }
       }
       if (more) {
+        if (next_q1) {
+          issue_qk(tmem + kColS1, dq(nb, 1), dk(st1), idesc_qk);
+          mma_commit(&sm.s_full[1]);
+        }
         mma_commit(&sm.k_empty[st1]);
-        if (j + 2 == x.nkv) mma_commit(&sm.q_empty[b]);
+        // release a Q buffer after the last QK that reads it
+        if (!last && j + 2 == x.nkv) mma_commit(&sm.q_empty[b]);
+        if (last && y.nkv == 1) mma_commit(&sm.q_empty[b2]);
       }
     }
-    if (!ok) break;
+    if (!ok || !has_next) break;
     kv_it += x.nkv;
     if (x.has_q1) { if (b) ++q1_it1; else ++q1_it0; }
+    x = y;
+    ++unit_it;
   }
   // All MMAs issued by this thread complete before TMEM is released.
   mma_commit(&sm.drain);
@@ -336,18 +418,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.q_full[0][i], 1);
-      mbar_init(&sm.q_full[1][i], 1);
+      for (int b = 0; b < kQBufs; ++b) {
+        mbar_init(&sm.q_full[b][i], 1);
+        mbar_init(&sm.q_ready[b][i], 1);
+      }
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i][0], kBM);
-      mbar_init(&sm.p_full[i][1], kBM);
+      for (int c = 0; c < kPChunks; ++c) mbar_init(&sm.p_full[i][c], kBM);
       mbar_init(&sm.o_done[i], 1);
     }
-    mbar_init(&sm.q_empty[0], 1);
-    mbar_init(&sm.q_empty[1], 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int b = 0; b < kQBufs; ++b) mbar_init(&sm.q_empty[b], 1);
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
@@ -359,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Ones chunk of every V stage: row r holds bf16 1.0 in column 0 and zeros elsewhere,
   // in the 64-byte swizzle the MMA reads (16-byte unit u of row r is stored at unit
   // u ^ ((r >> 1) & 3)).  TMA never writes this chunk.
-  for (int i = tid; i < kStages * 128 * 4; i += kThreads) {
+  for (int i = tid; i < kVStages * 128 * 4; i += kThreads) {
     const int st = i / (128 * 4), r = (i / 4) % 128, unit = i % 4;
     uint4 val = make_uint4(0u, 0u, 0u, 0u);
     if (unit == ((r >> 1) & 3)) val.x = 0x3F80u;  // bf16 1.0 in the low half = column 0
@@ -392,21 +476,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid() && ok;) {
         const Unit x = us.take();
         for (int j = 0; j < x.nkv; ++j, ++kv_it) {
-          const uint32_t st = kv_it % kStages, fill = kv_it / kStages;
+          const uint32_t sk = kv_it % kKStages, fk = kv_it / kKStages;
+          const uint32_t sv = kv_it % kVStages, fv = kv_it / kVStages;
           const int row0 = x.seg_start + j * kBN;
-          if (fill > 0 && !mbar_wait_bounded(&sm.k_empty[st], (fill - 1) & 1, abort_flag, dev_status)) {
+          if (fk > 0 && !mbar_wait_bounded(&sm.k_empty[sk], (fk - 1) & 1, abort_flag, dev_status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
-          tma_tile(sm.k[st], &tk, &sm.k_full[st], x.head, row0);
+          mbar_arrive_expect_tx(&sm.k_full[sk], kTileBytes);
+          tma_tile(sm.k[sk], &tk, &sm.k_full[sk], x.head, row0);
           ++k_issued;
-          if (fill > 0 && !mbar_wait_bounded(&sm.v_empty[st], (fill - 1) & 1, abort_flag, dev_status)) {
+          if (fv > 0 && !mbar_wait_bounded(&sm.v_empty[sv], (fv - 1) & 1, abort_flag, dev_status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&sm.v_full[st], kTileBytes);
-          tma_tile(sm.v[st], &tv, &sm.v_full[st], x.head, row0);
+          mbar_arrive_expect_tx(&sm.v_full[sv], kTileBytes);
+          tma_tile(sm.v[sv], &tv, &sm.v_full[sv], x.head, row0);
           ++v_issued;
         }
       }
@@ -414,12 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Every copy this thread issued has landed before the CTA exits.  Normally the MMA
         // thread has already waited on each of them and these waits return at once; after
         // an abort the last fills of the ring may still be in flight.  Only the last
-        // kStages fills per ring can be outstanding (each earlier one was waited on before
-        // its stage was refilled).
-        for (uint32_t f = (k_issued > kStages ? k_issued - kStages : 0); f < k_issued; ++f)
-          mbar_wait_drain(&sm.k_full[f % kStages], (f / kStages) & 1);
-        for (uint32_t f = (v_issued > kStages ? v_issued - kStages : 0); f < v_issued; ++f)
-          mbar_wait_drain(&sm.v_full[f % kStages], (f / kStages) & 1);
+        // fills of each ring (one per stage) can be outstanding (each earlier one was waited
+        // on before its stage was refilled).
+        for (uint32_t f = (k_issued > kKStages ? k_issued - kKStages : 0); f < k_issued; ++f)
+          mbar_wait_drain(&sm.k_full[f % kKStages], (f / kKStages) & 1);
+        for (uint32_t f = (v_issued > kVStages ? v_issued - kVStages : 0); f < v_issued; ++f)
+          mbar_wait_drain(&sm.v_full[f % kVStages], (f / kVStages) & 1);
       }
     }
    } else if (warp == kWarpLoadQ) {
@@ -429,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t unit_it = 0, q0a = 0, q0b = 0, q1a = 0, q1b = 0;
       for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid(); ++unit_it) {
         const Unit x = us.take();
-        const uint32_t b = unit_it & 1, use = unit_it >> 1;
+        const uint32_t b = unit_it % kQBufs, use = unit_it / kQBufs;
         // buffer b is free once every QK of the unit that used it before has completed
         if (use > 0 && !mbar_wait_bounded(&sm.q_empty[b], (use - 1) & 1, abort_flag, dev_status))
           break;
@@ -445,15 +530,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         // Every Q copy issued has landed before the CTA exits (see the K/V loader).
         if (q0a) mbar_wait_drain(&sm.q_full[0][0], (q0a - 1) & 1);
-        if (q0b) mbar_wait_drain(&sm.q_full[1][0], (q0b - 1) & 1);
         if (q1a) mbar_wait_drain(&sm.q_full[0][1], (q1a - 1) & 1);
-        if (q1b) mbar_wait_drain(&sm.q_full[1][1], (q1b - 1) & 1);
+        if (kQBufs > 1 && q0b) mbar_wait_drain(&sm.q_full[kQBufs - 1][0], (q0b - 1) & 1);
+        if (kQBufs > 1 && q1b) mbar_wait_drain(&sm.q_full[kQBufs - 1][1], (q1b - 1) & 1);
       }
     }
    } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       mma_role(sm, a, tmem, E, total, abort_flag, dev_status);
+    }
+   } else if (warp == kWarpRope && a.rope_pos != nullptr) {
+    // ------------------------------------------------------------ RoPE prologue of Q
+    // Each Q tile is rotated once, right after it lands; the loader runs a unit ahead, so
+    // this stays ahead of the QKs that read the tile (they wait on q_ready).  The Q buffer
+    // is only refilled after those QKs completed (q_empty), i.e. after this rotation.
+    uint32_t unit_it = 0, q1a = 0, q1b = 0;
+    for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid(); ++unit_it) {
+      const Unit x = us.take();
+      const uint32_t b = unit_it % kQBufs;
+      bool ok = true;
+      for (int i = 0; i < (x.has_q1 ? 2 : 1); ++i) {
+        const uint32_t parity = i == 0 ? (unit_it / kQBufs) & 1 : (b ? q1b : q1a) & 1;
+        if (!warp_wait(&sm.q_full[b][i], parity, abort_flag, dev_status)) { ok = false; break; }
+        rope_q_tile(sm.q[b][i], a.rope_pos, x.q0 + i * kBM, x.seg_end, a.rope.f, lane);
+        fence_proxy_async_smem();  // the rotated tile is read by the tensor core (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.q_ready[b][i]);
+      }
+      if (!ok) break;
+      if (x.has_q1) { if (b) ++q1b; else ++q1a; }
     }
    }
   } else {
@@ -478,9 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int nvalid = x.seg_end - (x.seg_start + j * kBN);  // >= 1
         const bool masked = nvalid < kBN;
+        float pm[8];
         // pass 1, row max: the row in two 64-column halves, eight independent
         // three-input max chains
-        float pm[8];
 #pragma unroll 1  // one copy of the half body: a smaller hot loop for the instruction cache
         for (int half = 0; half < 2; ++half) {
           uint32_t su[kBN / 2];

@@ -48,6 +48,15 @@ cudaError_t launch_schedule(const int32_t* cu_seqlens, int32_t num_segments, int
                             int32_t block_rows, WorkHeader* hdr, WorkEntry* entries,
                             cudaStream_t stream);
 
+// 2D RoPE frequencies f_i = theta^(-2 i / (D / 2)), i < D / 4, for D = 96 (host-computed).
+struct RopeFreqs {
+  float f[24];
+};
+RopeFreqs rope_freqs(double theta);
+// out = rope(x) for bf16 [T, H, 96] (out may equal x); pos: int32 [T][2] 1-based (pw, ph).
+cudaError_t launch_rope2d(const void* x, void* out, const int32_t* pos, int32_t T, int32_t H,
+                          const RopeFreqs& f, int num_sms, cudaStream_t stream);
+
 // bf16 forward on tcgen05 tensor cores (sm_100a).
 constexpr int kBf16BlockRows = 256;  // two 128-row Q tiles per unit
 struct Bf16Args {
@@ -63,6 +72,10 @@ struct Bf16Args {
   // > 0 only in the failure-path self-test: the MMA thread first waits this many cycles
   // on a barrier that never completes (see vt_attn_selftest_wait_timeout)
   int32_t stall_test_cycles = 0;
+  // 2D RoPE prologue: when rope_pos (device int32 [T][2], 1-based (pw, ph)) is set, every
+  // Q tile is rotated in shared memory after it lands and before any QK reads it
+  const int32_t* rope_pos = nullptr;
+  RopeFreqs rope;
 };
 size_t bf16_smem_bytes();
 cudaError_t prepare_attn_bf16();  // opt in to the kernel's dynamic shared memory (per device)
@@ -85,6 +98,37 @@ struct F32Args {
 size_t f32_smem_bytes();
 cudaError_t launch_attn_f32(const F32Args& args, int grid, cudaStream_t stream);
 
+// ---------------------------------------------------------------- host launcher
+// One forward call as the entry points receive it (validated by check_fwd_args).
+struct FwdCall {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  const int32_t* cu_seqlens;
+  int32_t num_segments, total_tokens, H;
+  float scale;
+  int dtype;  // vt_dtype
+  cudaStream_t stream;
+  int32_t stall_test_cycles;  // > 0 only for the bf16 failure-path self-test
+  const int32_t* rope_pos = nullptr;  // bf16 only: rotate Q by the 2D RoPE in the kernel
+  float rope_theta = 10000.0f;
+};
+
+// Host-side argument checks shared by every forward entry point; touches no device.
+// Returns 0 (VT_OK) or a vt_status code.  *no_work is set when the call is valid but
+// has nothing to compute (no segments, or no tokens).
+int check_fwd_args(const FwdCall& c, int32_t D, bool* no_work);
+
+// Query rows per work entry for a dtype (the kernel's unit of rows).
+int block_rows_for_dtype(int dtype);
+
+// Queues the scheduling prepass and the attention kernel of a validated call on
+// c.stream, with the work list at (hdr, entries) in device memory that holds at
+// least scratch_bytes_for(T, n, block_rows_for_dtype(dtype)) bytes.  The caller owns
+// that memory and orders its reuse.  Returns 0 or a vt_status code.
+int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries);
+
 // Window segmentation (window.cu).  Images are passed by value: at most kMaxWindowImages.
 constexpr int kMaxWindowImages = 64;
 struct WindowImages {
@@ -98,5 +142,8 @@ cudaError_t launch_window_perm(const WindowImages& g, int32_t* perm, int32_t* cu
 cudaError_t launch_permute_rows(const void* src, void* dst, const int32_t* idx, int32_t rows,
                                 int32_t row_bytes, int32_t scatter, int num_sms,
                                 cudaStream_t stream);
+// Reads, then clears, the device's out-of-range-index flag of launch_permute_rows
+// (synchronous; the current device).  *bad = 1 if some permute met such an index.
+cudaError_t permute_rows_check(int* bad);
 
 }  // namespace vt

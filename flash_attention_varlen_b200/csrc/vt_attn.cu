@@ -35,7 +35,8 @@ struct Scratch {
   size_t bytes = 0;
 };
 
-std::mutex g_mu;
+std::mutex g_mu;      // the per-stream work lists
+std::mutex g_dev_mu;  // the per-device launch information
 DeviceInfo g_dev[kMaxDevices];
 std::map<std::pair<int, uintptr_t>, Scratch> g_scratch;
 
@@ -145,92 +146,137 @@ size_t vt_attn_workspace_bytes(int32_t num_segments, int32_t total_tokens, vt_dt
 
 }  // extern "C"
 
-namespace {
+namespace vt {
 
-// The forward; stall_test_cycles > 0 only for the failure-path self-test (bf16).
-vt_status fwd_impl(const void* q, const void* k, const void* v, void* out,
-                   const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
-                   int32_t H, int32_t D, float scale, vt_dtype dtype, void* stream_ptr,
-                   int32_t stall_test_cycles) {
-  if (dtype != VT_DTYPE_BF16 && dtype != VT_DTYPE_F32) return VT_ERR_INVALID_ARG;
-  if (H < 1 || D < 1 || num_segments < 0 || total_tokens < 0) return VT_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return VT_ERR_INVALID_ARG;
+int block_rows_for_dtype(int dtype) { return block_rows_for(static_cast<vt_dtype>(dtype)); }
+
+int check_fwd_args(const FwdCall& c, int32_t D, bool* no_work) {
+  *no_work = false;
+  if (c.dtype != VT_DTYPE_BF16 && c.dtype != VT_DTYPE_F32) return VT_ERR_INVALID_ARG;
+  if (c.H < 1 || D < 1 || c.num_segments < 0 || c.total_tokens < 0) return VT_ERR_INVALID_ARG;
+  if (!std::isfinite(c.scale)) return VT_ERR_INVALID_ARG;
   if (D != kHeadDim) return VT_ERR_UNSUPPORTED;
-  if (num_segments == 0) return total_tokens == 0 ? VT_OK : VT_ERR_BAD_SEQLENS;
-  if (!cu_seqlens) return VT_ERR_NULL;
-  if (total_tokens == 0) return VT_OK;  // every segment is empty: nothing to write
-  if (!q || !k || !v || !out) return VT_ERR_NULL;
-  const uintptr_t align_or = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                             reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+  if (c.num_segments == 0) {
+    *no_work = true;
+    return c.total_tokens == 0 ? VT_OK : VT_ERR_BAD_SEQLENS;
+  }
+  if (!c.cu_seqlens) return VT_ERR_NULL;
+  if (c.total_tokens == 0) {  // every segment is empty: nothing to write
+    *no_work = true;
+    return VT_OK;
+  }
+  if (!c.q || !c.k || !c.v || !c.out) return VT_ERR_NULL;
+  const uintptr_t align_or = reinterpret_cast<uintptr_t>(c.q) | reinterpret_cast<uintptr_t>(c.k) |
+                             reinterpret_cast<uintptr_t>(c.v) | reinterpret_cast<uintptr_t>(c.out);
   if (align_or & 15u) return VT_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(H) * D > (1 << 20)) return VT_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) return VT_ERR_INVALID_ARG;
-  const size_t elem = dtype == VT_DTYPE_BF16 ? 2 : 4;
-  const size_t bytes = static_cast<size_t>(total_tokens) * H * D * elem;
-  if (ranges_overlap(out, bytes, q, bytes) || ranges_overlap(out, bytes, k, bytes) ||
-      ranges_overlap(out, bytes, v, bytes))
+  if (static_cast<int64_t>(c.H) * D > (1 << 20)) return VT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(c.cu_seqlens) & 3u) return VT_ERR_INVALID_ARG;
+  const size_t elem = c.dtype == VT_DTYPE_BF16 ? 2 : 4;
+  const size_t bytes = static_cast<size_t>(c.total_tokens) * c.H * D * elem;
+  if (ranges_overlap(c.out, bytes, c.q, bytes) || ranges_overlap(c.out, bytes, c.k, bytes) ||
+      ranges_overlap(c.out, bytes, c.v, bytes))
     return VT_ERR_INVALID_ARG;
+  return VT_OK;
+}
 
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-  std::lock_guard<std::mutex> lock(g_mu);
+int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return VT_ERR_CUDA;
   DeviceInfo* di = nullptr;
-  vt_status st = device_info(dev, &di);
-  if (st != VT_OK) return st;
-
-  const int block_rows = block_rows_for(dtype);
-  Scratch* sc = nullptr;
-  st = scratch_for(dev, stream, vt::scratch_bytes_for(total_tokens, num_segments, block_rows), &sc);
-  if (st != VT_OK) return st;
-  auto* hdr = static_cast<vt::WorkHeader*>(sc->ptr);
-  auto* entries = reinterpret_cast<vt::WorkEntry*>(hdr + 1);
-
-  if (vt::launch_schedule(cu_seqlens, num_segments, total_tokens, block_rows, hdr, entries,
-                          stream) != cudaSuccess)
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    vt_status st = device_info(dev, &di);
+    if (st != VT_OK) return st;
+    if (c.dtype == VT_DTYPE_BF16 && !di->bf16_ready) {
+      if (prepare_attn_bf16() != cudaSuccess) return VT_ERR_CUDA;
+      di->bf16_ready = true;
+    }
+  }
+  const int block_rows = block_rows_for_dtype(c.dtype);
+  if (launch_schedule(c.cu_seqlens, c.num_segments, c.total_tokens, block_rows, hdr, entries,
+                      c.stream) != cudaSuccess)
     return VT_ERR_CUDA;
 
   const long long max_units =
-      static_cast<long long>(vt::max_work_entries(total_tokens, num_segments, block_rows)) * H;
-  if (dtype == VT_DTYPE_BF16) {
-    if (!di->bf16_ready) {
-      if (vt::prepare_attn_bf16() != cudaSuccess) return VT_ERR_CUDA;
-      di->bf16_ready = true;
-    }
+      static_cast<long long>(max_work_entries(c.total_tokens, c.num_segments, block_rows)) * c.H;
+  if (c.dtype == VT_DTYPE_BF16) {
     CUtensorMap tq, tk, tv;
-    if ((st = make_tensor_map(&tq, q, total_tokens, H)) != VT_OK) return st;
-    if ((st = make_tensor_map(&tk, k, total_tokens, H)) != VT_OK) return st;
-    if ((st = make_tensor_map(&tv, v, total_tokens, H)) != VT_OK) return st;
-    vt::Bf16Args a;
-    a.out = out;
-    a.cu_seqlens = cu_seqlens;
+    vt_status st;
+    if ((st = make_tensor_map(&tq, c.q, c.total_tokens, c.H)) != VT_OK) return st;
+    if ((st = make_tensor_map(&tk, c.k, c.total_tokens, c.H)) != VT_OK) return st;
+    if ((st = make_tensor_map(&tv, c.v, c.total_tokens, c.H)) != VT_OK) return st;
+    Bf16Args a;
+    a.out = c.out;
+    a.cu_seqlens = c.cu_seqlens;
     a.hdr = hdr;
     a.entries = entries;
     a.dev_status = &hdr->status;
-    a.H = H;
-    a.out_align32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+    a.H = c.H;
+    a.out_align32 = (reinterpret_cast<uintptr_t>(c.out) & 31u) == 0;
     const double log2e = 1.4426950408889634;
-    a.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(scale)) * log2e);
-    a.idesc_qk = vt::make_idesc_bf16(128, 128, false, false, scale < 0.0f);
-    a.stall_test_cycles = stall_test_cycles;
+    a.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(c.scale)) * log2e);
+    a.idesc_qk = make_idesc_bf16(128, 128, false, false, c.scale < 0.0f);
+    a.stall_test_cycles = c.stall_test_cycles;
+    if (c.rope_pos != nullptr) {
+      a.rope_pos = c.rope_pos;
+      a.rope = rope_freqs(c.rope_theta);
+    }
     const int grid = static_cast<int>(max_units < di->num_sms ? max_units : di->num_sms);
-    if (vt::launch_attn_bf16(tq, tk, tv, a, grid, stream) != cudaSuccess) return VT_ERR_CUDA;
+    if (launch_attn_bf16(tq, tk, tv, a, grid, c.stream) != cudaSuccess) return VT_ERR_CUDA;
   } else {
-    vt::F32Args a;
-    a.q = static_cast<const float*>(q);
-    a.k = static_cast<const float*>(k);
-    a.v = static_cast<const float*>(v);
-    a.out = static_cast<float*>(out);
-    a.cu_seqlens = cu_seqlens;
+    F32Args a;
+    a.q = static_cast<const float*>(c.q);
+    a.k = static_cast<const float*>(c.k);
+    a.v = static_cast<const float*>(c.v);
+    a.out = static_cast<float*>(c.out);
+    a.cu_seqlens = c.cu_seqlens;
     a.hdr = hdr;
     a.entries = entries;
-    a.H = H;
-    a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    a.H = c.H;
+    a.scale_log2 = static_cast<float>(static_cast<double>(c.scale) * 1.4426950408889634);
     const long long cap = static_cast<long long>(di->num_sms) * 16;
     const int grid = static_cast<int>(max_units < cap ? max_units : cap);
-    if (vt::launch_attn_f32(a, grid, stream) != cudaSuccess) return VT_ERR_CUDA;
+    if (launch_attn_f32(a, grid, c.stream) != cudaSuccess) return VT_ERR_CUDA;
   }
   return VT_OK;
+}
+
+}  // namespace vt
+
+namespace {
+
+// The forward of a validated call with the library-owned, per-(device, stream) work list.
+vt_status fwd_impl(const vt::FwdCall& c) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  Scratch* sc = nullptr;
+  const vt_status st = scratch_for(dev, c.stream,
+                   vt::scratch_bytes_for(c.total_tokens, c.num_segments,
+                                         vt::block_rows_for_dtype(c.dtype)),
+                   &sc);
+  if (st != VT_OK) return st;
+  auto* hdr = static_cast<vt::WorkHeader*>(sc->ptr);
+  return static_cast<vt_status>(vt::launch_fwd(c, hdr, reinterpret_cast<vt::WorkEntry*>(hdr + 1)));
+}
+
+vt::FwdCall make_call(const void* q, const void* k, const void* v, void* out,
+                      const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                      int32_t H, float scale, vt_dtype dtype, void* stream_ptr, int32_t stall) {
+  vt::FwdCall c;
+  c.q = q;
+  c.k = k;
+  c.v = v;
+  c.out = out;
+  c.cu_seqlens = cu_seqlens;
+  c.num_segments = num_segments;
+  c.total_tokens = total_tokens;
+  c.H = H;
+  c.scale = scale;
+  c.dtype = dtype;
+  c.stream = static_cast<cudaStream_t>(stream_ptr);
+  c.stall_test_cycles = stall;
+  return c;
 }
 
 }  // namespace
@@ -240,8 +286,12 @@ extern "C" {
 vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
                       const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
                       int32_t H, int32_t D, float scale, vt_dtype dtype, void* stream_ptr) {
-  return fwd_impl(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D, scale, dtype,
-                  stream_ptr, 0);
+  vt::FwdCall c = make_call(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, scale, dtype,
+                            stream_ptr, 0);
+  bool no_work = false;
+  const vt_status st = static_cast<vt_status>(vt::check_fwd_args(c, D, &no_work));
+  if (st != VT_OK || no_work) return st;
+  return fwd_impl(c);
 }
 
 vt_status vt_attn_selftest_wait_timeout(const void* q, const void* k, const void* v, void* out,
@@ -250,8 +300,12 @@ vt_status vt_attn_selftest_wait_timeout(const void* q, const void* k, const void
                                         int32_t stall_cycles, void* stream_ptr) {
   if (stall_cycles < 1) return VT_ERR_INVALID_ARG;
   if (num_segments < 1 || total_tokens < 1) return VT_ERR_INVALID_ARG;  // a kernel must run
-  return fwd_impl(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D, scale,
-                  VT_DTYPE_BF16, stream_ptr, stall_cycles);
+  vt::FwdCall c = make_call(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, scale,
+                            VT_DTYPE_BF16, stream_ptr, stall_cycles);
+  bool no_work = false;
+  const vt_status st = static_cast<vt_status>(vt::check_fwd_args(c, D, &no_work));
+  if (st != VT_OK || no_work) return st;
+  return fwd_impl(c);
 }
 
 }  // extern "C"
@@ -336,6 +390,61 @@ vt_status vt_permute_rows(const void* src, void* dst, const int32_t* index, int3
              : VT_ERR_CUDA;
 }
 
+vt_status vt_attn_fwd_rope2d(const void* q, const void* k, const void* v, void* out,
+                             const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                             int32_t H, int32_t D, float scale, const int32_t* pos, float theta,
+                             void* k_rot, void* stream_ptr) {
+  vt::FwdCall c = make_call(q, k_rot, v, out, cu_seqlens, num_segments, total_tokens, H, scale,
+                            VT_DTYPE_BF16, stream_ptr, 0);
+  bool no_work = false;
+  vt_status st = static_cast<vt_status>(vt::check_fwd_args(c, D, &no_work));
+  if (st != VT_OK || no_work) return st;
+  if (!std::isfinite(theta) || !(theta > 0.0f)) return VT_ERR_INVALID_ARG;
+  if (!k || !pos) return VT_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(k) & 15u) || (reinterpret_cast<uintptr_t>(pos) & 7u))
+    return VT_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(total_tokens) * H * D * 2;
+  if (k != k_rot && (ranges_overlap(k, bytes, k_rot, bytes) || ranges_overlap(k, bytes, out, bytes)))
+    return VT_ERR_INVALID_ARG;
+  if (ranges_overlap(k_rot, bytes, q, bytes) || ranges_overlap(k_rot, bytes, v, bytes))
+    return VT_ERR_INVALID_ARG;
+  // K is rotated once by the HBM-bound pass (each K tile is read by every unit of its
+  // segment, so rotating it there would repeat the work per unit); Q is rotated inside the
+  // attention kernel, once per unit, after its tile lands in shared memory.
+  st = vt_rope2d(k, k_rot, pos, total_tokens, H, D, theta, stream_ptr);
+  if (st != VT_OK) return st;
+  c.rope_pos = pos;
+  c.rope_theta = theta;
+  return fwd_impl(c);
+}
+
+vt_status vt_rope2d(const void* x, void* out, const int32_t* pos, int32_t total_tokens, int32_t H,
+                    int32_t D, float theta, void* stream) {
+  if (H < 1 || D < 1 || total_tokens < 0) return VT_ERR_INVALID_ARG;
+  if (!std::isfinite(theta) || !(theta > 0.0f)) return VT_ERR_INVALID_ARG;
+  if (D != kHeadDim) return VT_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return VT_OK;
+  if (!x || !out || !pos) return VT_ERR_NULL;
+  if (((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15u) ||
+      (reinterpret_cast<uintptr_t>(pos) & 7u))
+    return VT_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(total_tokens) * H * D * 2;
+  if (x != out && ranges_overlap(x, bytes, out, bytes)) return VT_ERR_INVALID_ARG;
+  const int nsm = sm_count();
+  if (nsm < 1) return VT_ERR_CUDA;
+  return vt::launch_rope2d(x, out, pos, total_tokens, H, vt::rope_freqs(theta), nsm,
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? VT_OK
+             : VT_ERR_CUDA;
+}
+
+vt_status vt_permute_rows_check(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return VT_ERR_CUDA;
+  int bad = 0;
+  if (vt::permute_rows_check(&bad) != cudaSuccess) return VT_ERR_CUDA;
+  return bad ? VT_ERR_BAD_INDEX : VT_OK;
+}
+
 vt_status vt_attn_last_device_status(void* stream_ptr) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   int dev = 0;
@@ -365,6 +474,7 @@ const char* vt_attn_status_string(vt_status s) {
     case VT_ERR_BAD_SEQLENS: return "VT_ERR_BAD_SEQLENS: cu_seqlens must start at 0, not decrease and end at total_tokens";
     case VT_ERR_CUDA: return "VT_ERR_CUDA: a CUDA call failed";
     case VT_ERR_DEVICE_TIMEOUT: return "VT_ERR_DEVICE_TIMEOUT: a kernel pipeline wait gave up";
+    case VT_ERR_BAD_INDEX: return "VT_ERR_BAD_INDEX: a row index outside [0, num_rows) was skipped";
   }
   return "unknown vt_status";
 }

@@ -1,8 +1,9 @@
 // Window segmentation on the device: the permutation that makes each win x win block of
 // an image's patch grid a contiguous segment, its cu_seqlens, and a row gather/scatter.
 //
-// The vision tower attends within windows of 32 x 32 patches in its window layers (PR #279,
-// "Two of the three labelled uncertainties are now resolved").  Its hidden states are put
+// The vision tower attends within windows of 32 x 32 patches in its window layers (issue
+// #1545 (vllm.cpp), follow-up comment, the section on the resolved labelled uncertainties:
+// the window side comes from the positional-embedding grid).  Its hidden states are put
 // in window order once, before the first layer, and back in image order once, after the
 // last (PR #279, vision-tower port commit: the inverse permutation comes before ln_post and
 // the RoPE table is permuted alongside).  So the attention kernel reads packed, contiguous
@@ -58,8 +59,14 @@ __global__ void window_perm_kernel(const WindowImages g, int32_t* __restrict__ p
   }
 }
 
+// Set (never cleared by a kernel) when a permute met an index outside [0, rows); the host
+// reads and clears it (permute_rows_check).  One word per device, shared by all calls.
+__device__ int g_permute_bad_index;
+
 // dst[i] = src[idx[i]] (gather) or dst[idx[i]] = src[i] (scatter), rows of row_bytes
-// (a multiple of 16), one warp per row, 16-byte accesses.
+// (a multiple of 16), one warp per row, 16-byte accesses.  A row whose index lies outside
+// [0, rows) is skipped before any access (nothing read or written for it) and raises the
+// device's flag, so a bad index from the caller cannot reach outside the two buffers.
 __global__ void permute_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                     const int32_t* __restrict__ idx, int32_t rows,
                                     int32_t row_vec, int32_t scatter) {
@@ -68,6 +75,10 @@ __global__ void permute_rows_kernel(const uint4* __restrict__ src, uint4* __rest
   for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
        r += warps) {
     const int64_t j = __ldg(idx + r);
+    if (j < 0 || j >= rows) {
+      if (lane == 0) atomicOr(&g_permute_bad_index, 1);
+      continue;
+    }
     const int64_t s = scatter ? r : j, d = scatter ? j : r;
     const uint4* sp = src + s * row_vec;
     uint4* dp = dst + d * row_vec;
@@ -76,6 +87,18 @@ __global__ void permute_rows_kernel(const uint4* __restrict__ src, uint4* __rest
 }
 
 }  // namespace
+
+cudaError_t permute_rows_check(int* bad) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_permute_bad_index, sizeof(int));
+  if (e != cudaSuccess) return e;
+  *bad = v;
+  if (v) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_permute_bad_index, &zero, sizeof(int));
+  }
+  return e;
+}
 
 cudaError_t launch_window_perm(const WindowImages& g, int32_t* perm, int32_t* cu,
                                int num_sms, cudaStream_t stream) {

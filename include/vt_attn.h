@@ -22,7 +22,10 @@
  * allocated on the first call on that stream and grown (never shrunk) when a
  * call needs more; make a first call on a stream before capturing it in a
  * CUDA graph.  Calls are stream-ordered; calls on different streams use
- * different scratch buffers.
+ * different scratch buffers.  The library keeps per-device state (launch
+ * attributes, work lists, device addresses) for the life of the device's primary
+ * context: a cudaDeviceReset invalidates it, so do not call the library again in a
+ * process after resetting a device it has used.
  *
  * Errors: every entry point returns a status and never throws or aborts.
  * Argument errors are detected on the host before anything is launched.
@@ -52,7 +55,8 @@ typedef enum {
   VT_ERR_UNSUPPORTED = 3,    /* a valid request the library does not implement (D != 96) */
   VT_ERR_BAD_SEQLENS = 4,    /* cu_seqlens not 0 = cu[0] <= ... <= cu[n] = total_tokens */
   VT_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed */
-  VT_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up waiting on its own pipeline (bug guard) */
+  VT_ERR_DEVICE_TIMEOUT = 6, /* a kernel gave up waiting on its own pipeline (bug guard) */
+  VT_ERR_BAD_INDEX = 7       /* vt_permute_rows met a row index outside [0, num_rows) */
 } vt_status;
 
 /*
@@ -97,8 +101,11 @@ vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
  *     anything);
  *   - every call on a device shares the array, so calls that may overlap on the
  *     GPU (e.g. on two streams) race and must be serialised by the caller;
- *   - a malformed cu_seqlens makes the call write nothing; it is not reported by
- *     vt_attn_last_device_status, which covers vt_attn_fwd's own work lists.
+ *   - what the device side finds is not reported: vt_attn_last_device_status covers
+ *     vt_attn_fwd's own work lists only.  A malformed cu_seqlens makes the call write
+ *     nothing; a kernel wait that gives up (VT_ERR_DEVICE_TIMEOUT for vt_attn_fwd, a
+ *     guard against a broken pipeline, never expected) leaves `out` partly written
+ *     without a report.  Callers that need these checks use vt_attn_fwd.
  */
 vt_status vt_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
                               const int32_t* cu_seqlens, int32_t num_segments,
@@ -107,7 +114,12 @@ vt_status vt_attn_fwd_noalloc(const void* q, const void* k, const void* v, void*
 
 /*
  * Pure host check of a host copy of cu_seqlens (num_segments+1 entries):
- * VT_OK, VT_ERR_NULL or VT_ERR_BAD_SEQLENS.  Touches no GPU.
+ * VT_OK, VT_ERR_NULL or VT_ERR_BAD_SEQLENS.  Touches no GPU.  The segments are the
+ * block-diagonal mask as contiguous row slices (issue #1545 (vllm.cpp), "The fix"),
+ * so they must tile [0, total_tokens): cu[0] = 0, non-decreasing, cu[n] =
+ * total_tokens.  The check covers the whole array before any loop relies on it (PR
+ * #279, vision-tower port commit: a coverage check placed after the slicing loop let
+ * a bad input hang instead of fail).
  */
 vt_status vt_attn_validate_seqlens_host(const int32_t* cu_seqlens_host, int32_t num_segments,
                                         int32_t total_tokens);
@@ -159,10 +171,11 @@ vt_status vt_attn_selftest_wait_timeout(const void* q, const void* k, const void
 
 /*
  * Window segmentation (the vision tower's window layers attend within 32 x 32-patch
- * windows of each image: PR #279, "Two of the three labelled uncertainties are now
- * resolved").  The tower puts its hidden states in window order once before its layers
- * and back in image order once after them (PR #279, vision-tower port commit).  The
- * calls below build that order on the device and apply it to [rows, ...] tensors.
+ * windows of each image: issue #1545 (vllm.cpp), follow-up comment, the section on the
+ * resolved labelled uncertainties).  The tower puts its hidden states in window order
+ * once before its layers and back in image order once after them (PR #279,
+ * vision-tower port commit).  The calls below build that order on the device and apply
+ * it to [rows, ...] tensors.
  *
  * Order (the pages name the two orders without printing them; the plain row-major
  * reading):
@@ -195,10 +208,64 @@ vt_status vt_window_partition(const int32_t* grids, int32_t n_images, int32_t wi
  * to window order with index = perm); scatter == 1 scatters dst[index[i]] = src[i]
  * (back).  Rows are row_bytes long (a multiple of 16, e.g. H * D * 2 for bf16
  * [T, H, D]); src and dst are device pointers, 16-byte aligned, and must not overlap;
- * index holds num_rows distinct row numbers in [0, num_rows).
+ * index holds num_rows distinct row numbers in [0, num_rows).  index lives on the
+ * device, so its values are checked there: a row whose index lies outside
+ * [0, num_rows) is skipped before any memory access (gather: dst row i keeps its
+ * contents; scatter: nothing is written for it) and raises a per-device flag that
+ * vt_permute_rows_check reports.
  */
 vt_status vt_permute_rows(const void* src, void* dst, const int32_t* index, int32_t num_rows,
                           int32_t row_bytes, int32_t scatter, void* stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the current device's out-of-range
+ * flag of vt_permute_rows: VT_ERR_BAD_INDEX if any vt_permute_rows call on this device
+ * since the previous check skipped a row (on any stream: the flag is one word per
+ * device), else VT_OK; VT_ERR_CUDA if the synchronisation or the read failed.
+ */
+vt_status vt_permute_rows_check(void* stream);
+
+/*
+ * 2D rotary position embedding of the vision tower: out = rope(x) for a bf16
+ * [total_tokens, H, D] tensor (PR #279, vision-tower port commit: the tower rotates Q and
+ * K by a width-first 2D RoPE with 1-based positions, and the RoPE table travels with the
+ * hidden states into window order).  The pages print no formula; the reading taken:
+ *   pos        device int32 [total_tokens][2]: (pw, ph) = (x + 1, y + 1), the token's
+ *              1-based column and row in its image's patch grid (in window order when the
+ *              tokens are, e.g. gathered with vt_permute_rows);
+ *   f_i        = theta^(-2 i / (D / 2)), i < D / 4 (computed on the host in double);
+ *   angle a_d  = pw * f_d for d < D/4, ph * f_{d - D/4} for D/4 <= d < D/2 (width first);
+ *   element d < D/2 pairs with d + D/2: (x_d, x_{d+D/2}) turns by a_d.
+ * Arithmetic in f32 (sin/cos after reduction to [-pi, pi]); the result is rounded to bf16.
+ *   x, out   device pointers, 16-byte aligned; out == x rotates in place, otherwise the
+ *            two must not overlap.
+ *   D        only 96 (VT_ERR_UNSUPPORTED otherwise); H >= 1; theta finite and > 0 (the
+ *            tower's base: 10000).
+ * Asynchronous on `stream`; total_tokens == 0 is a no-op.
+ */
+vt_status vt_rope2d(const void* x, void* out, const int32_t* pos, int32_t total_tokens, int32_t H,
+                    int32_t D, float theta, void* stream);
+
+/*
+ * Attention with the vision tower's 2D RoPE applied to Q and K first:
+ *     O = attention(rope(Q), rope(K), V)   per segment, as vt_attn_fwd,
+ * with rope() exactly as vt_rope2d defines it (bf16 only; D = 96).
+ *   pos     device int32 [total_tokens][2], the tokens' 1-based (pw, ph) (in the same
+ *           order as q, k, v: window order for a window layer).
+ *   theta   RoPE base, finite and > 0 (the tower's: 10000).
+ *   k_rot   caller-owned device buffer [total_tokens, H, D] bf16, 16-byte aligned, that
+ *           receives rope(K) (the attention reads K from it); k_rot == k rotates K in
+ *           place.  It must not overlap q, v or out.
+ * Q is rotated inside the attention kernel: each 128-row Q tile once, in shared memory,
+ * right after it lands and before the QK products read it (the fused RoPE prologue).  K
+ * is rotated by one HBM-bound vt_rope2d pass queued first on the same stream: every K tile
+ * is read by all units of its segment, so rotating it inside the kernel would repeat the
+ * rotation once per unit.  Errors and asynchrony as for vt_attn_fwd.
+ */
+vt_status vt_attn_fwd_rope2d(const void* q, const void* k, const void* v, void* out,
+                             const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                             int32_t H, int32_t D, float scale, const int32_t* pos, float theta,
+                             void* k_rot, void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* vt_attn_status_string(vt_status status);
