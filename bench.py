@@ -319,7 +319,8 @@ def run_ours(args):
 
     # the other configurations of the workload, one layer each (informational): after the
     # timed region, on this rank's GPU
-    configs = time_configs(fa, torch, dev) if not args.no_configs else None
+    outputs = {} if (rank == 0 and not args.no_cpu_baseline) else None
+    configs = time_configs(fa, torch, dev, keep_outputs=outputs) if not args.no_configs else None
 
     result = {
         "metric": METRIC,
@@ -368,6 +369,9 @@ def run_ours(args):
     }
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = oracle_sample(args.cpu_seconds)
+        if configs:
+            for name, entry in oracle_per_config(outputs).items():
+                configs[name]["vs_oracle"] = entry
     if distributed:
         dist.barrier()
         dist.destroy_process_group()
@@ -375,11 +379,52 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3):
+def config_cases():
+    return [workloads.tiny_case("bf16"), workloads.tiny_case("f32"), workloads.image448_case(),
+            workloads.image448_case(True), *workloads.image896_cases(), workloads.varlen8_case()]
+
+
+def bf16_round(x):
+    """f64 values rounded to the nearest bf16 (ties to even), kept in f64."""
+    x = np.asarray(x, np.float64)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126))) - 7)
+    return np.round(x / ulp) * ulp
+
+
+def oracle_per_config(outputs):
+    """CPU-baseline leg, per configuration: the oracle (f64, all host cores) timed on each
+    configuration's whole input, and the GPU output's error against it: max/mean-abs, the
+    max-abs against the oracle rounded to bf16 (the output's own rounding floor), and
+    max |O|.  Runs after the timed region; `outputs` maps a configuration name to
+    (case, GPU output as f64)."""
+    import oracle
+    threads = oracle.default_threads()
+    res = {}
+    for name, (c, got) in outputs.items():
+        q, k, v = c.inputs()
+        t0 = time.perf_counter()
+        ref = oracle.attn_fwd(q, k, v, c.cu_seqlens, SCALE, threads=threads)
+        dt = time.perf_counter() - t0
+        err = np.abs(got - ref)
+        entry = {"max_abs": float(err.max()), "mean_abs": float(err.mean()),
+                 "max_abs_O": float(np.abs(ref).max()), "finite": bool(np.isfinite(got).all()),
+                 "oracle_s": round(dt, 3), "oracle_tflops": round(c.flops() / dt / 1e12, 5),
+                 "cores": threads}
+        if c.dtype == "bf16":
+            entry["max_abs_vs_bf16_oracle"] = float(np.abs(got - bf16_round(ref)).max())
+            entry["within_bound"] = bool(err.max() <= 1e-2 and err.mean() <= 1e-3)
+        else:
+            entry["within_bound"] = bool(err.max() <= 1e-5)
+        res[name] = entry
+    return res
+
+
+def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3, keep_outputs=None):
     """ms per call and TFLOP/s of each smaller configuration of the workload (one layer, the
-    inputs resident; calls back to back, so these small cases run partly out of L2)."""
-    cases = [workloads.tiny_case("bf16"), workloads.tiny_case("f32"), workloads.image448_case(),
-             workloads.image448_case(True), *workloads.image896_cases(), workloads.varlen8_case()]
+    inputs resident; calls back to back, so these small cases run partly out of L2).  With
+    `keep_outputs` (a dict), each configuration's output is stored there, as f64 on the host,
+    for the error check after the timed region."""
+    cases = config_cases()
     stream = torch.cuda.current_stream(dev)
     out = {}
     for c in cases:
@@ -412,6 +457,8 @@ def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3):
         ms = e0.elapsed_time(e1) / calls
         out[c.name] = {"dtype": c.dtype, "segments": c.num_segments, "tokens": c.T,
                        "ms": round(ms, 4), "tflops": round(c.flops() / (ms * 1e-3) / 1e12, 2)}
+        if keep_outputs is not None:
+            keep_outputs[c.name] = (c, do.float().cpu().numpy().astype(np.float64))
     try:  # informational: must never cost the headline line
         out["window_segmentation_128x128"] = time_window_segmentation(fa, torch, dev, calls)
     except Exception as exc:  # noqa: BLE001
@@ -575,8 +622,20 @@ def run_single_layer(args):
                       "calls": args.steps, "note": "back-to-back calls on one layer's inputs"}))
 
 
+def check_world(args):
+    """--gpus N must match the number of ranks launched (torchrun sets WORLD_SIZE; a plain
+    `python bench.py` is one rank): N replicas come from torchrun, never from this flag."""
+    _, world, _ = rank_info()
+    if args.gpus != world:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but {world} rank(s) were launched; run "
+                         f"`python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py "
+                         f"--gpus {args.gpus} ...` for more than one GPU\n")
+        sys.exit(2)
+
+
 def main(argv=None):
     args = parse_args(argv)
+    check_world(args)
     if args.single_layer:
         run_single_layer(args)
     elif args.impl == "reference":

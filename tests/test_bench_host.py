@@ -46,3 +46,16 @@ def test_fingerprint_follows_code(tmp_path):
 def test_current_kernel_fingerprint_is_well_formed():
     fp = bench.kernel_sha()
     assert len(fp) == 16 and int(fp, 16) >= 0
+
+
+def test_gpus_flag_must_match_the_launched_ranks(monkeypatch, capsys):
+    """`--gpus N` is only honoured through torchrun's WORLD_SIZE; a mismatch is refused
+    instead of silently running one replica."""
+    import pytest
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    bench.check_world(bench.parse_args(["--gpus", "1"]))  # one rank, as launched
+    with pytest.raises(SystemExit) as e:
+        bench.check_world(bench.parse_args(["--gpus", "8"]))
+    assert e.value.code == 2 and "--gpus 8" in capsys.readouterr().err
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    bench.check_world(bench.parse_args(["--gpus", "4"]))

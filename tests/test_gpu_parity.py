@@ -115,10 +115,41 @@ def test_varlen8_images():
     _sampled_case(workloads.varlen8_case(), n_rows=4096)
 
 
+def _unit_rows(cu, H, seed, rows_per_entry=256):
+    """One (token, head) row in every work unit the bf16 kernel runs (256 query rows of one
+    segment and head), placed so that over the units every (Q tile, 32-lane TMEM quarter)
+    of a unit is covered: offset ((entry + head) % 8) * 32 + a random lane, clipped to the
+    segment."""
+    rng = np.random.default_rng(seed)
+    tok, head = [], []
+    entry = 0
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        for r0 in range(a, b, rows_per_entry):
+            n = min(rows_per_entry, b - r0)
+            for h in range(H):
+                off = ((entry + h) % 8) * 32 + int(rng.integers(0, 32))
+                tok.append(r0 + min(off, n - 1))
+                head.append(h)
+            entry += 1
+    return np.array(tok, np.int32), np.array(head, np.int32)
+
+
 def test_tower16k_every_layer():
-    """All 50 layers of the 16384-token tower, as the benchmark runs them, on sampled rows."""
+    """All 50 layers of the 16384-token tower, as the benchmark runs them: one row in every
+    (256-row entry, head) unit of every layer (1024 rows per layer), covering both Q tiles
+    and all four TMEM lane quarters of a unit."""
     for case in workloads.tower_cases():
-        _sampled_case(case, n_rows=96, seed=case.seed)
+        q, k, v = case.inputs()
+        got = _run(q, k, v, case.cu_seqlens, "bf16")
+        tok, head = _unit_rows(case.cu_seqlens, case.H, case.seed)
+        ref = oracle.attn_rows(q, k, v, case.cu_seqlens, SCALE, tok, head)
+        _check(got[tok, head], ref, "bf16", case.name)
+
+
+def test_tower16k_window_layer_in_full():
+    """Layer 0 of the tower (16 windows of 1024 tokens) compared element by element."""
+    _full_case(workloads.tower_layer_case(0))
 
 
 # ---------------------------------------------------------------- edge cases
@@ -152,32 +183,83 @@ def test_other_head_counts(dtype, H):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("scale", [0.0, -0.1, 0.15])
+@pytest.mark.parametrize("scale", [0.0, -0.25, -0.1, 0.15])
 def test_scales(dtype, scale):
-    """Zero (uniform attention) and negative scales, at logit spreads like the encoder's."""
+    """Zero (uniform attention) and negative scales, at logit spreads up to ~2.5x the
+    encoder's (scale -0.25: logit std ~2.5), under the fixed bounds."""
     case = workloads.Case(f"scale_{dtype}", workloads.cu_from_lengths([200, 333]), seed=5, dtype=dtype)
     _full_case(case, scale=scale)
 
 
-def test_very_peaked_rows_bf16_representation_floor():
+def _bf16_round(x):
+    """Round f64 values to the nearest bf16 (ties to even), in f64."""
+    x = np.asarray(x, np.float64)
+    mag = np.maximum(np.abs(x), 2.0 ** -126)
+    ulp = np.exp2(np.floor(np.log2(mag)) - 7)
+    return np.round(x / ulp) * ulp
+
+
+def bf16_floor_report(got, ref):
+    """Error against the oracle and against the oracle rounded to bf16, max |O|, and the
+    elements over the 1e-2 bound that neither have |O| >= 4 nor equal the bf16-rounded
+    oracle to within half an ulp (the output-rounding floor)."""
+    err = np.abs(got - ref)
+    rb = _bf16_round(ref)
+    err_rb = np.abs(got - rb)
+    half_ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(rb), 2.0 ** -126))) - 8)
+    over = err > BF16_MAX
+    unexplained = over & ~((np.abs(ref) >= 4.0) | (err_rb <= half_ulp))
+    return {"max_abs": float(err.max()), "mean_abs": float(err.mean()),
+            "max_abs_vs_bf16_oracle": float(err_rb.max()), "max_abs_O": float(np.abs(ref).max()),
+            "over_bound": int(over.sum()), "unexplained": int(unexplained.sum())}
+
+
+def test_scale_half_bf16_bound_or_output_rounding_floor():
     """scale 0.5 on N(0,1) data: logit std ~4.9, rows close to one-hot, |O| up to ~4.
 
-    Here bf16 output rounding alone costs up to half an ulp (2^-7 = 7.8e-3 for
-    |O| in [2, 4)), and P is a bf16 operand of the PV product, so the fixed
-    1e-2 bound is not the right yardstick.  Checked instead: error <= half an ulp
-    of the output plus 2^-9 * max|V| (one bf16 rounding of the dominant weight),
-    and the f32 arm at its usual 1e-5.
+    The fixed bounds still apply (mean-abs <= 1e-3, max-abs <= 1e-2), except where the
+    bf16 output itself cannot meet them: an element over 1e-2 must have |O| >= 4 (half
+    an ulp there is 1.6e-2) or be the oracle rounded to bf16 to within half an ulp.  The
+    f32 arm meets its usual 1e-5 on the same rows.
     """
     case = workloads.Case("peaked05", workloads.cu_from_lengths([200, 333]), seed=5, dtype="bf16")
     q, k, v = case.inputs()
     got = _run(q, k, v, case.cu_seqlens, "bf16", scale=0.5)
     ref = oracle.attn_fwd(q, k, v, case.cu_seqlens, 0.5)
-    half_ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 8)
-    vmax = np.abs(workloads.bf16_bits_to_f32(v)).max()
-    assert np.all(np.abs(got - ref) <= half_ulp + 2.0 ** -9 * vmax)
-    assert np.abs(got - ref).mean() <= BF16_MEAN
+    rep = bf16_floor_report(got, ref)
+    print("scale 0.5 bf16:", rep)
+    assert np.isfinite(got).all()
+    assert rep["mean_abs"] <= BF16_MEAN, rep
+    assert rep["unexplained"] == 0, rep
     case32 = workloads.Case("peaked05_f32", case.cu_seqlens, seed=5, dtype="f32")
     _full_case(case32, scale=0.5)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_scores_far_below_the_running_max(dtype):
+    """Every other key of each segment sits ~300 binades below its row's running max (so
+    its exp2 argument reaches the polynomial's clamp and the MUFU's flush to zero); the
+    other keys form an ordinary softmax.  Exactly, the far keys' weights are below
+    2^-290 of the max, so the result is attention over the near keys, and the oracle,
+    computing in f64 on the same inputs, resolves it.  Component 0 carries the split:
+    q_0 = 16 for every row, k_0 = -128 for the far keys (both exact in bf16)."""
+    lengths = [300, 129, 1000, 2]
+    cu = workloads.cu_from_lengths(lengths)
+    case = workloads.Case(f"far_{dtype}", cu, seed=12, dtype=dtype)
+    q, k, v = case.inputs()
+    f32 = (lambda a: workloads.bf16_bits_to_f32(a)) if dtype == "bf16" else (lambda a: a)
+    qf, kf = f32(q).copy(), f32(k).copy()
+    qf[:, :, 0] = 16.0
+    kf[1::2, :, 0] = -128.0
+    if dtype == "bf16":
+        q, k = (np.ascontiguousarray(a).view(np.uint32) >> 16 for a in (qf, kf))
+        q, k = q.astype(np.uint16), k.astype(np.uint16)
+        assert np.array_equal(workloads.bf16_bits_to_f32(k), kf)  # the values were bf16 already
+    else:
+        q, k = qf, kf
+    got = _run(q, k, v, cu, dtype)
+    ref = oracle.attn_fwd(q, k, v, cu, SCALE)
+    _check(got, ref, dtype, case.name)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])

@@ -72,3 +72,38 @@ def test_window_layer_from_image_order(grids):
     err = np.abs(got - ref)
     assert np.isfinite(got).all()
     assert err.max() <= 1e-2 and err.mean() <= 1e-3
+
+
+@pytest.mark.parametrize("inverse", [False, True], ids=["gather", "scatter"])
+def test_permute_rows_skips_out_of_range_indexes(inverse):
+    """index lives on the device, so the kernel checks it: rows whose index is outside
+    [0, T) are skipped before any access (no fault) and reported by the check call;
+    every other row moves exactly as numpy indexing says."""
+    import flash_attention_varlen_b200 as fa
+    from flash_attention_varlen_b200 import _binding as b
+    T = 1000
+    fa.check_permute_rows()  # start from a clear flag
+    g = torch.Generator().manual_seed(3)
+    p = torch.randperm(T, generator=g).to(torch.int32)
+    bad_rows = [5, 611, 999]
+    p[5], p[611], p[999] = T, -1, 2 ** 31 - 1
+    x = torch.randn(T, 16, 96, generator=g).to(torch.bfloat16).cuda()
+    out = torch.full_like(x, 3.0)
+    fa.permute_rows(x, p.cuda(), inverse=inverse, out=out)
+    with pytest.raises(fa.VtAttnError) as e:
+        fa.check_permute_rows()
+    assert e.value.status == b.VT_ERR_BAD_INDEX
+    fa.check_permute_rows()  # reading cleared the flag
+    got, xs = out.cpu(), x.cpu()
+    good = [i for i in range(T) if i not in bad_rows]
+    pl = p.long()
+    if inverse:
+        assert torch.equal(got[pl[good]], xs[good])
+        untouched = sorted(set(range(T)) - set(pl[good].tolist()))
+        assert untouched and torch.all(got[untouched] == 3.0)
+    else:
+        assert torch.equal(got[good], xs[pl[good]])
+        assert torch.all(got[bad_rows] == 3.0)
+    # a valid permutation afterwards reports nothing
+    fa.permute_rows(x, torch.randperm(T, generator=g).to(torch.int32).cuda(), inverse=inverse)
+    fa.check_permute_rows()
