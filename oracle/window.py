@@ -4,9 +4,9 @@ Only ``tests/`` (and ``bench.py``'s CPU legs) may import this; the CUDA library 
 does, and the two share no code.
 
 The vision tower's window layers attend within windows of 32 x 32 = 1024 patches of each
-image's patch grid (PR #279, "Two of the three labelled uncertainties are now resolved":
-pos_emb_height and pos_emb_width are both 32, and the tower's sparse permutation segments
-the grid on them).  The pages name the permutation's two orders, the walk over the blocks
+image's patch grid (issue #1545 (vllm.cpp), follow-up comment, the section on the
+resolved labelled uncertainties: the positional-embedding grid is 32 x 32, and the
+tower's sparse permutation segments the patch grid on it).  The pages name the permutation's two orders, the walk over the blocks
 and the order of the tokens inside a block, as places a port goes wrong (PR #279, vision
 tower port commit), but print neither.  The plainest reading is taken here:
   * images are packed one after another, each in row-major (y, x) patch order;

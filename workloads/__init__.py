@@ -14,8 +14,9 @@ width 96 (issue #1545 "Why this one is bad": H=16, head_dim=96), 448x448 and
 896x896 images at patch 14 (1024 and 4096 patch tokens), 32x32-patch windows
 (issue #1545 follow-up: pos_emb_height = pos_emb_width = 32) and a 50-layer
 schedule whose full-attention layers sit at indices 3, 7, 11, ..., 47, 49, the
-other 37 being window layers (issue #1545 follow-up, "Two of the three labelled
-uncertainties are now resolved").  The 128x128-patch grid is the issue's
+other 37 being window layers (issue #1545 follow-up comment, the section on the
+resolved labelled uncertainties: the split is read from the shipped configuration).
+The 128x128-patch grid is the issue's
 "reading A" (16384 patch tokens, 16 windows).
 """
 from __future__ import annotations
