@@ -2,8 +2,8 @@
 
 The rotation pass computes in f32 (angles pos * f_i, reduced to [-pi, pi], hardware sin/cos
 with ~2^-21 absolute error) and rounds to bf16, so each element is compared with the f64
-oracle within one bf16 ulp of the oracle's value (the output rounding, plus a margin far
-larger than the f32 arithmetic error).  Positions are those of the tower's 128 x 128 patch
+oracle within one bf16 ulp of the oracle's value (the output rounding) plus a bound on the
+f32 evaluation error, which grows with the angle (two f32 roundings of pos * f_i).  Positions are those of the tower's 128 x 128 patch
 grid taken in window order, as the tower carries them.
 """
 import numpy as np
@@ -30,15 +30,17 @@ def _bf16_dev(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def _within_one_ulp(got, ref, x):
-    """|got - ref| <= one bf16 ulp of ref plus the f32 evaluation's absolute error: the
-    hardware sin/cos err by ~2^-21 on the reduced angle and each output element is
-    x_d cos - x_{d+48} sin (or the mirror), so 2^-19 (|x_d| + |x_{d+48}|) bounds it; it
-    matters where the two terms cancel and ref, hence its ulp, is tiny."""
+def _within_one_ulp(got, ref, x, ang):
+    """|got - ref| <= one bf16 ulp of ref plus the f32 evaluation's absolute error.  The
+    f32 angle pos * f_i carries two roundings (f_i and the product), under |a| 2^-23; the
+    reduction and the hardware sin/cos add ~2^-21; each output element is
+    x_d cos - x_{d+48} sin (or the mirror), so (|x_d| + |x_{d+48}|)(|a| 2^-22 + 2^-20) bounds
+    it with a factor of two to spare.  It matters where the two terms cancel and ref, hence
+    its ulp, is tiny."""
     ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
     pair = np.abs(x[..., :48]) + np.abs(x[..., 48:])
-    eps = 2.0 ** -19 * np.concatenate([pair, pair], axis=-1)
-    return np.abs(got - ref) <= ulp + eps
+    err = pair * (np.abs(ang)[:, None, :] * 2.0 ** -22 + 2.0 ** -20)
+    return np.abs(got - ref) <= ulp + np.concatenate([err, err], axis=-1)
 
 
 def tower_positions(grid=128, win=32):
@@ -56,10 +58,16 @@ def test_rope2d_matches_oracle_on_the_tower_grid(theta):
     torch.cuda.synchronize()
     got = got.float().cpu().numpy().astype(np.float64)
     ref = rope.rope2d(q, pos, theta)
-    ok = _within_one_ulp(got, ref, workloads.bf16_bits_to_f32(q).astype(np.float64))
+    ang = rope.rope_angles(pos, 96, theta)
+    ok = _within_one_ulp(got, ref, workloads.bf16_bits_to_f32(q).astype(np.float64), ang)
     assert np.isfinite(got).all() and ok.all(), f"{(~ok).sum()} elements beyond one ulp"
-    # and mostly the correctly rounded value itself
-    assert np.mean(np.abs(got - ref)) < 2.0 ** -10
+    # and almost everywhere the correctly rounded oracle value itself: the f32 error only
+    # flips the rounding of values within ~2^-16 relative of a rounding midpoint
+    b = ref.astype(np.float32).view(np.uint32)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16 << 16).astype(np.uint32)
+    ref_bf16 = b.view(np.float32).astype(np.float64)
+    assert np.mean(got == ref_bf16) > 0.99
+    assert np.mean(np.abs(got - ref)) <= 1.01 * np.mean(np.abs(ref_bf16 - ref))
 
 
 def test_rope2d_in_place_equals_out_of_place_and_position_zero_is_identity():
