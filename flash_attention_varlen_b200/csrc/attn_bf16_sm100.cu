@@ -100,6 +100,15 @@ __device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, volatil
   return mbar_wait_bounded(bar, parity, abort_flag, dev_status);
 }
 
+// The work list of a call with at most kInlineSegments segments, built in shared memory
+// by the kernel itself (no prepass): its segments longest first, each as
+// (segment, 0, start, end), and the prefix sums of their entry counts.
+struct SchedTable {
+  int4 seg[kInlineSegments];
+  int32_t prefix[kInlineSegments + 1];
+  int32_t n, E, order, bad;
+};
+
 struct Smem {
   uint8_t q[kQBufs][2][kTileBytes];
   uint8_t k[kKStages][kTileBytes];
@@ -118,6 +127,7 @@ struct Smem {
   uint64_t never;  // nothing arrives on it: the failure-path self-test waits here
   uint32_t tmem_base;
   int abort_flag;
+  SchedTable sched;
 };
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
@@ -141,14 +151,15 @@ struct Unit {
 //    stride over head-major units left some with twice the mean).
 // Each unit is decoded from its 16-byte entry, and the next unit's entry is loaded as soon
 // as the current one is taken, so that load's latency is hidden behind a whole unit of
-// work instead of stalling every role at each unit boundary.  The unit count stays below
-// 2^31 (tokens x heads in device memory).
+// work instead of stalling every role at each unit boundary.  With a shared-memory work
+// table (a call of few segments) the entry is looked up there instead.  The unit count
+// stays below 2^31 (tokens x heads in device memory).
 class UnitStream {
  public:
-  __device__ __forceinline__ UnitStream(const WorkEntry* entries, uint32_t E, uint32_t total,
-                                        uint32_t H, int order)
-      : entries_(reinterpret_cast<const int4*>(entries)), E_(E), H_(H), total_(total),
-        entry_major_(order != 0) {
+  __device__ __forceinline__ UnitStream(const WorkEntry* entries, const SchedTable* tab,
+                                        uint32_t E, uint32_t total, uint32_t H, int order)
+      : entries_(reinterpret_cast<const int4*>(entries)), tab_(tab), E_(E), H_(H),
+        total_(total), entry_major_(order != 0) {
     locate();
   }
   __device__ __forceinline__ bool valid() const { return u_ < total_; }
@@ -178,9 +189,18 @@ class UnitStream {
       head_ = u_ / E_;
       e = u_ - head_ * E_;
     }
-    cur_ = __ldg(entries_ + e);
+    if (tab_ != nullptr) {  // the last segment whose first entry is <= e
+      int s = 0;
+#pragma unroll 1
+      while (s + 1 < tab_->n && tab_->prefix[s + 1] <= static_cast<int>(e)) ++s;
+      cur_ = tab_->seg[s];
+      cur_.y = static_cast<int>(e) - tab_->prefix[s];
+    } else {
+      cur_ = __ldg(entries_ + e);
+    }
   }
   const int4* entries_;
+  const SchedTable* tab_;
   uint32_t E_, H_, total_, k_ = 0, u_ = 0, head_ = 0;
   bool entry_major_;
   int4 cur_ = make_int4(0, 0, 0, 0);
@@ -287,11 +307,68 @@ __device__ __forceinline__ void rope_q_tile(uint8_t* tile, const int32_t* pos, i
   }
 }
 
+// Builds the shared-memory work table of a call with n <= kInlineSegments segments, by one
+// warp: the same validation (cu[0] == 0, cu[n] == T, no negative length), the same
+// longest-first order (ties by index) and the same unit order flag as the scheduling
+// prepass, so the units, and the results, are identical to that path's.
+__device__ __forceinline__ void build_sched_table(SchedTable& t, const int32_t* cu, int n, int T,
+                                                  int lane) {
+  constexpr unsigned kAll = 0xffffffffu;
+  int start = 0, end = 0;
+  bool bad = false;
+  if (lane < n) {
+    start = __ldg(cu + lane);
+    end = __ldg(cu + lane + 1);
+    bad = end < start || (lane == 0 && start != 0) || (lane == n - 1 && end != T);
+  }
+  bad = __any_sync(kAll, bad);
+  const int len = end - start;
+  // key = (INT_MAX - len) << 32 | segment: ascending order = longest first
+  unsigned long long key =
+      lane < n ? (static_cast<unsigned long long>(0x7FFFFFFFu - static_cast<unsigned>(len)) << 32) |
+                     static_cast<unsigned>(lane)
+               : ~0ull;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {  // bitonic sort over the warp, ascending
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(kAll, key, j);
+      const bool keep_min = ((lane & j) == 0) == ((lane & k) == 0);
+      key = keep_min ? (other < key ? other : key) : (other < key ? key : other);
+    }
+  }
+  const int seg = lane < n ? static_cast<int>(key & 0xFFFFFFFFu) : 0;  // at sorted position lane
+  const int ss = __shfl_sync(kAll, start, seg), se = __shfl_sync(kAll, end, seg);
+  const int cnt = lane < n ? (se - ss + kBf16BlockRows - 1) / kBf16BlockRows : 0;
+  int incl = cnt;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(kAll, incl, d);
+    if (lane >= d) incl += y;
+  }
+  const int E = __shfl_sync(kAll, incl, n - 1);
+  // segments of unequal (non-empty) lengths: entry-major order, longest first
+  const int lmin = __reduce_min_sync(kAll, lane < n && len > 0 ? len : 0x7FFFFFFF);
+  const int lmax = __reduce_max_sync(kAll, lane < n && len > 0 ? len : 0);
+  if (lane < n) {
+    t.seg[lane] = make_int4(seg, 0, ss, se);
+    t.prefix[lane + 1] = incl;
+  }
+  if (lane == 0) {
+    t.prefix[0] = 0;
+    t.n = n;
+    t.bad = bad ? 1 : 0;
+    t.E = bad ? 0 : E;
+    t.order = lmin < lmax ? 1 : 0;
+  }
+}
+
 // The MMA issuer (one thread).  It is kept out of line so that its loop is one compact
 // piece of code: the thread sleeps in mbarrier waits between short bursts of MMA
 // issue, and its wake-up latency is on the critical path of every key tile.
-__device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem, uint32_t E, uint32_t total,
-                                      volatile int* abort_flag, int* dev_status) {
+__device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem, const SchedTable* tab,
+                                      uint32_t E, uint32_t total, int order, volatile int* abort_flag,
+                                      int* dev_status) {
   if (a.stall_test_cycles > 0) {
     // Failure-path self-test: this wait can never succeed, so it runs out after
     // stall_test_cycles, raises the CTA's abort flag and records a timeout; every other
@@ -326,7 +403,7 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
   // where tile j+1 after a unit's last tile is the next unit's first.  So a Q tile's next S
   // is computed right after its own last PV of a unit (during that tile's epilogue), not
   // behind the other tile's last PV.  The K/V ring runs on across units as the loader fills it.
-  UnitStream us(a.entries, E, total, a.H, a.hdr->order);
+  UnitStream us(a.entries, tab, E, total, a.H, order);
   bool ok = us.valid();
   Unit x;
   if (ok) {
@@ -412,10 +489,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (raw & 1023u)) & 1023u));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t E = static_cast<uint32_t>(a.hdr->num_entries);
-  const uint32_t total = E * static_cast<uint32_t>(a.H);
-  if (blockIdx.x >= total) return;  // uniform over the CTA
 
+  // Set-up that reads nothing the scheduling prepass writes: with programmatic dependent
+  // launch it overlaps the prepass.
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       for (int b = 0; b < kQBufs; ++b) {
@@ -466,6 +542,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &sm.abort_flag;
   int* dev_status = a.dev_status;
 
+  // Inputs and the work list are read only after the previous kernel in the stream (the
+  // prepass, when one runs) has completed.
+  griddep_wait();
+  const SchedTable* tab = nullptr;
+  uint32_t E;
+  int order;
+  if (a.inline_sched) {
+    if (warp == 0) build_sched_table(sm.sched, a.cu_seqlens, a.num_segments, a.total_tokens, lane);
+    __syncthreads();
+    tab = &sm.sched;
+    E = static_cast<uint32_t>(sm.sched.E);
+    order = sm.sched.order;
+    if (blockIdx.x == 0 && tid == 0) {
+      *a.next_status = 0;  // the next call on this scratch starts after this one ends
+      if (sm.sched.bad) atomicOr(a.dev_status, kDevStatusBadSeqlens);
+    }
+  } else {
+    E = static_cast<uint32_t>(a.hdr->num_entries);
+    order = a.hdr->order;
+  }
+  const uint32_t total = E * static_cast<uint32_t>(a.H);
+  if (blockIdx.x >= total) {  // uniform over the CTA: no unit for it
+    if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+    return;
+  }
+
   if (warp >= 8) {
    setmaxnreg_dec<kRegsOther>();
    if (warp == kWarpLoad) {
@@ -473,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kv_it = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
-      for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid() && ok;) {
+      for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid() && ok;) {
         const Unit x = us.take();
         for (int j = 0; j < x.nkv; ++j, ++kv_it) {
           const uint32_t sk = kv_it % kKStages, fk = kv_it / kKStages;
@@ -512,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // per-buffer load counts (kept in scalars: a runtime-indexed array would go to local memory)
       uint32_t unit_it = 0, q0a = 0, q0b = 0, q1a = 0, q1b = 0;
-      for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid(); ++unit_it) {
+      for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid(); ++unit_it) {
         const Unit x = us.take();
         const uint32_t b = unit_it % kQBufs, use = unit_it / kQBufs;
         // buffer b is free once every QK of the unit that used it before has completed
@@ -538,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
    } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      mma_role(sm, a, tmem, E, total, abort_flag, dev_status);
+      mma_role(sm, a, tmem, tab, E, total, order, abort_flag, dev_status);
     }
    } else if (warp == kWarpRope && a.rope_pos != nullptr) {
     // ------------------------------------------------------------ RoPE prologue of Q
@@ -546,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // this stays ahead of the QKs that read the tile (they wait on q_ready).  The Q buffer
     // is only refilled after those QKs completed (q_empty), i.e. after this rotation.
     uint32_t unit_it = 0, q1a = 0, q1b = 0;
-    for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid(); ++unit_it) {
+    for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid(); ++unit_it) {
       const Unit x = us.take();
       const uint32_t b = unit_it % kQBufs;
       bool ok = true;
@@ -572,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + (wg ? kColO1 : kColO0);
     const float c = a.scale_log2;
     uint32_t s_cnt = 0, o_base = 0;
-    for (UnitStream us(a.entries, E, total, a.H, a.hdr->order); us.valid();) {
+    for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid();) {
       const Unit x = us.take();
       if (wg == 1 && !x.has_q1) continue;
       const int row_tok = x.q0 + wg * kBM + r;
@@ -738,8 +840,19 @@ size_t bf16_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const Bf16Args& args, int grid, cudaStream_t stream) {
-  attn_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, args);
-  return cudaGetLastError();
+  // Programmatic stream serialization: the kernel may launch while the scheduling prepass
+  // before it still runs, and waits for it (griddepcontrol.wait) before reading its output.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_bf16_kernel, tq, tk, tv, args);
 }
 
 cudaError_t prepare_attn_bf16() {

@@ -7,17 +7,21 @@
 
 namespace vt {
 
-// Head of the per-stream scratch buffer, written by the scheduling prepass.
+// Head of the per-stream scratch buffer.
 struct alignas(128) WorkHeader {
-  int32_t status;       // kDevStatus* bit flags of the last call on this scratch
-  int32_t num_entries;  // E: number of (segment, q-block) entries that follow
+  // kDevStatus* bit flags, one word per call parity: the call with slot k reports what
+  // its device side finds in status[k] and clears status[k ^ 1], the word of the next
+  // call on the same scratch, before that call can start
+  int32_t status[2];
+  int32_t num_entries;  // E: number of (segment, q-block) entries that follow (prepass)
   // Unit order of the bf16 kernel, set by the prepass: 0 = head-major (unit u = head u / E,
   // entry u % E), for segments of one length: the CTAs in flight share few heads' K/V in
   // L2; 1 = entry-major (entry u / H, head u % H), for segments of unequal length: the
   // units come longest first, which the snake assignment needs to balance the CTAs
   int32_t order;
-  int32_t pad[29];
+  int32_t pad[28];
 };
+static_assert(sizeof(WorkHeader) == 128, "header size");
 
 // A work entry: one block of `block_rows` query rows of one segment, stored
 // decoded (the segment's bounds included) so a kernel reads it with a single
@@ -42,11 +46,16 @@ inline size_t scratch_bytes_for(int64_t total_tokens, int64_t num_segments, int 
 }
 
 // Scheduling prepass (one CTA): validates cu_seqlens, orders segments by
-// length (longest first) and writes the entry list.  Sets status to
-// kDevStatusBadSeqlens and num_entries to 0 on a malformed cu_seqlens.
+// length (longest first) and writes the entry list.  Sets status[slot] to 0, or to
+// kDevStatusBadSeqlens with num_entries 0 on a malformed cu_seqlens, and clears
+// status[slot ^ 1].
 cudaError_t launch_schedule(const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
-                            int32_t block_rows, WorkHeader* hdr, WorkEntry* entries,
+                            int32_t block_rows, int slot, WorkHeader* hdr, WorkEntry* entries,
                             cudaStream_t stream);
+
+// The bf16 kernel builds the work list of a call with at most this many segments itself,
+// in shared memory (same validation and order as the prepass), and no prepass runs.
+constexpr int kInlineSegments = 32;
 
 // 2D RoPE frequencies f_i = theta^(-2 i / (D / 2)), i < D / 4, for D = 96 (host-computed).
 struct RopeFreqs {
@@ -64,7 +73,10 @@ struct Bf16Args {
   const int32_t* cu_seqlens;
   const WorkHeader* hdr;
   const WorkEntry* entries;
-  int* dev_status;
+  int* dev_status;   // this call's status word
+  int* next_status;  // the next call's status word (cleared by this call when inline)
+  int32_t num_segments, total_tokens;
+  int32_t inline_sched;  // 1: no prepass ran; the kernel builds the work list itself
   int32_t H;
   int32_t out_align32;  // out is 32-byte aligned: rows go out as 256-bit stores
   float scale_log2;    // |scale| * log2(e)
@@ -127,7 +139,9 @@ int block_rows_for_dtype(int dtype);
 // c.stream, with the work list at (hdr, entries) in device memory that holds at
 // least scratch_bytes_for(T, n, block_rows_for_dtype(dtype)) bytes.  The caller owns
 // that memory and orders its reuse.  Returns 0 or a vt_status code.
-int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries);
+// `slot` (0 or 1) is the call's status word in hdr; successive calls on one scratch
+// alternate it.
+int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot);
 
 // Window segmentation (window.cu).  Images are passed by value: at most kMaxWindowImages.
 constexpr int kMaxWindowImages = 64;

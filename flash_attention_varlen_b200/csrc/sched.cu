@@ -30,12 +30,15 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
 
 __global__ void __launch_bounds__(kThreads)
     schedule_kernel(const int32_t* __restrict__ cu, int32_t n, int32_t T, int32_t block_rows,
-                    WorkHeader* hdr, WorkEntry* entries) {
+                    int slot, WorkHeader* hdr, WorkEntry* entries) {
   __shared__ unsigned long long keys[kSortMax];
   __shared__ int warp_sums[32];
   __shared__ int chunk_total;
   __shared__ int len_min, len_max;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // The attention kernel that follows may launch now and set itself up while this runs;
+  // it reads the work list only after this grid has completed.
+  griddep_launch_dependents();
   if (tid == 0) {
     len_min = 0x7FFFFFFF;
     len_max = 0;
@@ -55,7 +58,8 @@ __global__ void __launch_bounds__(kThreads)
   }
   if (__syncthreads_or(bad)) {
     if (tid == 0) {
-      hdr->status = kDevStatusBadSeqlens;
+      hdr->status[slot] = kDevStatusBadSeqlens;
+      hdr->status[slot ^ 1] = 0;
       hdr->num_entries = 0;
       hdr->order = 0;
     }
@@ -139,17 +143,18 @@ __global__ void __launch_bounds__(kThreads)
   if (tid == 0) {
     hdr->num_entries = base;
     hdr->order = (do_sort && len_min < len_max) ? 1 : 0;  // unequal lengths: longest first
-    hdr->status = 0;
+    hdr->status[slot] = 0;
+    hdr->status[slot ^ 1] = 0;
   }
 }
 
 }  // namespace
 
 cudaError_t launch_schedule(const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
-                            int32_t block_rows, WorkHeader* hdr, WorkEntry* entries,
+                            int32_t block_rows, int slot, WorkHeader* hdr, WorkEntry* entries,
                             cudaStream_t stream) {
   schedule_kernel<<<1, kThreads, 0, stream>>>(cu_seqlens, num_segments, total_tokens, block_rows,
-                                              hdr, entries);
+                                              slot, hdr, entries);
   return cudaGetLastError();
 }
 

@@ -33,6 +33,8 @@ struct DeviceInfo {
 struct Scratch {
   void* ptr = nullptr;
   size_t bytes = 0;
+  uint32_t calls = 0;  // forward calls queued on this scratch: their status slots alternate
+  int last_slot = 0;   // status slot of the latest one
 };
 
 std::mutex g_mu;      // the per-stream work lists
@@ -179,7 +181,7 @@ int check_fwd_args(const FwdCall& c, int32_t D, bool* no_work) {
   return VT_OK;
 }
 
-int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries) {
+int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return VT_ERR_CUDA;
   DeviceInfo* di = nullptr;
@@ -193,8 +195,10 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries) {
     }
   }
   const int block_rows = block_rows_for_dtype(c.dtype);
-  if (launch_schedule(c.cu_seqlens, c.num_segments, c.total_tokens, block_rows, hdr, entries,
-                      c.stream) != cudaSuccess)
+  // A bf16 call with few segments needs no prepass: its kernel builds the work list.
+  const bool inline_sched = c.dtype == VT_DTYPE_BF16 && c.num_segments <= kInlineSegments;
+  if (!inline_sched && launch_schedule(c.cu_seqlens, c.num_segments, c.total_tokens, block_rows,
+                                       slot, hdr, entries, c.stream) != cudaSuccess)
     return VT_ERR_CUDA;
 
   const long long max_units =
@@ -210,7 +214,11 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries) {
     a.cu_seqlens = c.cu_seqlens;
     a.hdr = hdr;
     a.entries = entries;
-    a.dev_status = &hdr->status;
+    a.dev_status = &hdr->status[slot];
+    a.next_status = &hdr->status[slot ^ 1];
+    a.num_segments = c.num_segments;
+    a.total_tokens = c.total_tokens;
+    a.inline_sched = inline_sched ? 1 : 0;
     a.H = c.H;
     a.out_align32 = (reinterpret_cast<uintptr_t>(c.out) & 31u) == 0;
     const double log2e = 1.4426950408889634;
@@ -257,7 +265,10 @@ vt_status fwd_impl(const vt::FwdCall& c) {
                    &sc);
   if (st != VT_OK) return st;
   auto* hdr = static_cast<vt::WorkHeader*>(sc->ptr);
-  return static_cast<vt_status>(vt::launch_fwd(c, hdr, reinterpret_cast<vt::WorkEntry*>(hdr + 1)));
+  const int slot = static_cast<int>(sc->calls++ & 1u);
+  sc->last_slot = slot;
+  return static_cast<vt_status>(
+      vt::launch_fwd(c, hdr, reinterpret_cast<vt::WorkEntry*>(hdr + 1), slot));
 }
 
 vt::FwdCall make_call(const void* q, const void* k, const void* v, void* out,
@@ -449,16 +460,16 @@ vt_status vt_attn_last_device_status(void* stream_ptr) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return VT_ERR_CUDA;
-  void* ptr = nullptr;
+  const int32_t* word = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     auto it = g_scratch.find({dev, reinterpret_cast<uintptr_t>(stream)});
     if (it == g_scratch.end() || !it->second.ptr) return VT_OK;
-    ptr = it->second.ptr;
+    word = static_cast<const vt::WorkHeader*>(it->second.ptr)->status + it->second.last_slot;
   }
   if (cudaStreamSynchronize(stream) != cudaSuccess) return VT_ERR_CUDA;
   int status = 0;
-  if (cudaMemcpy(&status, ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaMemcpy(&status, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return VT_ERR_CUDA;
   if (status & vt::kDevStatusBadSeqlens) return VT_ERR_BAD_SEQLENS;
   if (status & vt::kDevStatusTimeout) return VT_ERR_DEVICE_TIMEOUT;

@@ -38,6 +38,7 @@ struct NoAllocDevice {
 
 std::mutex g_noalloc_mu;
 NoAllocDevice g_noalloc_dev[kMaxDevicesNoAlloc];
+uint32_t g_noalloc_calls[kMaxDevicesNoAlloc];  // calls per device: their status slots alternate
 
 // Per-device set-up on the first call made with that device current: the device address
 // of the array.  In host code the name g_noalloc_scratch is only a host-side stand-in, so
@@ -93,5 +94,7 @@ extern "C" vt_status vt_attn_fwd_noalloc(const void* q, const void* k, const voi
   void* scratch = nullptr;
   if ((st = noalloc_scratch(dev, &scratch)) != VT_OK) return st;
   auto* hdr = static_cast<vt::WorkHeader*>(scratch);
-  return static_cast<vt_status>(vt::launch_fwd(c, hdr, reinterpret_cast<vt::WorkEntry*>(hdr + 1)));
+  const int slot = static_cast<int>(g_noalloc_calls[dev]++ & 1u);  // status slots alternate
+  return static_cast<vt_status>(
+      vt::launch_fwd(c, hdr, reinterpret_cast<vt::WorkEntry*>(hdr + 1), slot));
 }
