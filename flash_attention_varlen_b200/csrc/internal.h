@@ -94,20 +94,22 @@ cudaError_t prepare_attn_bf16();  // opt in to the kernel's dynamic shared memor
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const Bf16Args& args, int grid, cudaStream_t stream);
 
-// f32 forward on FP32 FMA pipes (exactness arm).
-constexpr int kF32BlockRows = 64;
+// f32 forward on tcgen05 tensor cores: each operand split into three bf16 parts
+// (exactness arm).
+constexpr int kF32BlockRows = 128;
 struct F32Args {
   const float* q;
   const float* k;
   const float* v;
   float* out;
-  const int32_t* cu_seqlens;
   const WorkHeader* hdr;
   const WorkEntry* entries;
-  int32_t H;
+  int* dev_status;
+  int32_t H, T;
   float scale_log2;  // scale * log2(e), signed
 };
 size_t f32_smem_bytes();
+cudaError_t prepare_attn_f32();  // opt in to the kernel's dynamic shared memory (per device)
 cudaError_t launch_attn_f32(const F32Args& args, int grid, cudaStream_t stream);
 
 // ---------------------------------------------------------------- host launcher

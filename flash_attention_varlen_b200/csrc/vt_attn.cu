@@ -28,6 +28,7 @@ struct DeviceInfo {
   bool init = false;
   int num_sms = 0;
   bool bf16_ready = false;
+  bool f32_ready = false;
 };
 
 struct Scratch {
@@ -61,8 +62,8 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-// [T, H, 96] bf16 viewed as (d, h, t); a box is 32 columns x 1 head x 128 rows,
-// stored with the 64-byte swizzle the MMA descriptors expect.
+// [T, H, 96] bf16 viewed as (d, h, t); a box is 32 columns x 1 head x 128 rows, stored
+// with the 64-byte swizzle (32 columns = 64 bytes per row) the MMA descriptors expect.
 vt_status make_tensor_map(CUtensorMap* map, const void* base, int32_t T, int32_t H) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return VT_ERR_CUDA;
@@ -193,6 +194,10 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) 
       if (prepare_attn_bf16() != cudaSuccess) return VT_ERR_CUDA;
       di->bf16_ready = true;
     }
+    if (c.dtype == VT_DTYPE_F32 && !di->f32_ready) {
+      if (prepare_attn_f32() != cudaSuccess) return VT_ERR_CUDA;
+      di->f32_ready = true;
+    }
   }
   const int block_rows = block_rows_for_dtype(c.dtype);
   // A bf16 call with few segments needs no prepass: its kernel builds the work list.
@@ -237,13 +242,13 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) 
     a.k = static_cast<const float*>(c.k);
     a.v = static_cast<const float*>(c.v);
     a.out = static_cast<float*>(c.out);
-    a.cu_seqlens = c.cu_seqlens;
     a.hdr = hdr;
     a.entries = entries;
+    a.dev_status = &hdr->status[slot];
     a.H = c.H;
+    a.T = c.total_tokens;
     a.scale_log2 = static_cast<float>(static_cast<double>(c.scale) * 1.4426950408889634);
-    const long long cap = static_cast<long long>(di->num_sms) * 16;
-    const int grid = static_cast<int>(max_units < cap ? max_units : cap);
+    const int grid = static_cast<int>(max_units < di->num_sms ? max_units : di->num_sms);
     if (launch_attn_f32(a, grid, c.stream) != cudaSuccess) return VT_ERR_CUDA;
   }
   return VT_OK;
