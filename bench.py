@@ -358,7 +358,7 @@ def run_ours(args):
             "frac": round(achieved / peak, 4),
             "peak_source": f"{peak_src} dense bf16 (MEASURED_PEAKS.json bf16_tflops)",
             "traffic": traffic,
-            "kernel": "attn_bf16_kernel (+ its scheduling prepass, timed together per call)",
+            "kernel": "attn_bf16_kernel (calls of at most 32 segments, as in the tower, schedule themselves; a prepass would be timed with its call)",
             "per_launch": "4*sum(L^2)*H*D FLOPs of the call / CUDA-event duration of the call, "
                           "averaged FLOP-weighted over the 50 calls of a step",
         },

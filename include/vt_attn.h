@@ -45,7 +45,8 @@ extern "C" {
 
 typedef enum {
   VT_DTYPE_BF16 = 0, /* bfloat16 inputs/outputs, f32 accumulation (tensor cores) */
-  VT_DTYPE_F32 = 1   /* float32 inputs/outputs, f32 arithmetic (FMA pipes) */
+  VT_DTYPE_F32 = 1   /* float32 inputs/outputs, within 1e-5 of exact: tensor cores on
+                        operands split into three bf16 parts, f32 softmax */
 } vt_dtype;
 
 typedef enum {

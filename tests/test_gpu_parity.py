@@ -342,6 +342,14 @@ def test_long_single_segment():
     _sampled_case(case, n_rows=256)
 
 
+@pytest.mark.parametrize("scale", [SCALE, -0.25])
+def test_long_f32_segments_keep_the_f32_bound(scale):
+    """The f32 arm sums PV per 64-key tile and folds the tiles into O in f32; a 4096-token
+    segment (64 key tiles) and a 1000-token one next to it, sampled rows at 1e-5."""
+    case = workloads.Case("long_f32", workloads.cu_from_lengths([4096, 1000]), seed=12, dtype="f32")
+    _sampled_case(case, n_rows=512, scale=scale)
+
+
 def test_empty_inputs_are_noops():
     import flash_attention_varlen_b200 as fa
     z = torch.zeros(0, 16, 96, dtype=torch.bfloat16, device="cuda")
