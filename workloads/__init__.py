@@ -160,6 +160,38 @@ def flops(cu_seqlens, H: int = HEADS, D: int = HEAD_DIM) -> int:
     return int(4 * int((L * L).sum()) * H * D)
 
 
+# Text decoder attention (the Muse Glimmer next-steps document, "Architecture / Text
+# decoder"): 32 query heads over 2 key/value heads, head size 128, local window 2048.
+DECODER_HQ, DECODER_HKV, DECODER_D, DECODER_WINDOW = 32, 2, 128, 2048
+
+
+def decoder_qkv(seed: int, T: int, Hq: int = DECODER_HQ, Hkv: int = DECODER_HKV,
+                D: int = DECODER_D, dtype: str = "bf16"):
+    """Q [T, Hq, D], K and V [T, Hkv, D] from streams 0, 1, 2 of ``seed``."""
+    q = normal(seed, STREAM_Q, T * Hq * D, dtype).reshape(T, Hq, D)
+    k = normal(seed, STREAM_K, T * Hkv * D, dtype).reshape(T, Hkv, D)
+    v = normal(seed, STREAM_V, T * Hkv * D, dtype).reshape(T, Hkv, D)
+    return q, k, v
+
+
+def decoder_pairs(cu_seqlens, window: int) -> int:
+    """(query, key) pairs of causal attention with a local window (0: none), per head: query
+    n (1-based within its segment) sees min(n, window) keys."""
+    cu = np.asarray(cu_seqlens, np.int64)
+    total = 0
+    for L in (cu[1:] - cu[:-1]).tolist():
+        if window <= 0 or window >= L:
+            total += L * (L + 1) // 2
+        else:
+            total += window * (window + 1) // 2 + (L - window) * window
+    return int(total)
+
+
+def decoder_flops(cu_seqlens, window: int, Hq: int = DECODER_HQ, D: int = DECODER_D) -> int:
+    """Algorithmic FLOPs of the decoder attention forward: 4 * pairs * Hq * D."""
+    return 4 * decoder_pairs(cu_seqlens, window) * Hq * D
+
+
 def exp_count(cu_seqlens, H: int = HEADS) -> int:
     """Softmax exponentials of one forward: sum(L^2) * H (one per score)."""
     cu = np.asarray(cu_seqlens, np.int64)
