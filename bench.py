@@ -400,7 +400,11 @@ def oracle_per_config(outputs):
     import oracle
     threads = oracle.default_threads()
     res = {}
-    for name, (c, got) in outputs.items():
+    for name, item in outputs.items():
+        if item[0] == "decoder":
+            res[name] = decoder_vs_oracle(*item[1:])
+            continue
+        c, got = item
         q, k, v = c.inputs()
         t0 = time.perf_counter()
         ref = oracle.attn_fwd(q, k, v, c.cu_seqlens, SCALE, threads=threads)
@@ -417,6 +421,26 @@ def oracle_per_config(outputs):
             entry["within_bound"] = bool(err.max() <= 1e-5)
         res[name] = entry
     return res
+
+
+def decoder_vs_oracle(inputs, got):
+    """The decoder output against its oracle on one row of every 128-row block of each
+    query head, alternating ends of the block: errors, max |O| and the oracle's time."""
+    from oracle import decoder
+    q, k, v, cu, window, scale = inputs
+    T, Hq = q.shape[0], q.shape[1]
+    blocks = np.arange(0, T, 128)
+    tok = np.concatenate([blocks + (h % 2) * 127 for h in range(Hq)])
+    head = np.repeat(np.arange(Hq), len(blocks))
+    t0 = time.perf_counter()
+    ref = decoder.attn_rows(q, k, v, cu, scale, window, tok, head)
+    dt = time.perf_counter() - t0
+    err = np.abs(got[tok, head] - ref)
+    return {"rows": int(len(tok)), "max_abs": float(err.max()), "mean_abs": float(err.mean()),
+            "max_abs_O": float(np.abs(ref).max()), "finite": bool(np.isfinite(got).all()),
+            "max_abs_vs_bf16_oracle": float(np.abs(got[tok, head] - bf16_round(ref)).max()),
+            "within_bound": bool(err.max() <= 1e-2 and err.mean() <= 1e-3),
+            "oracle_s_rows": round(dt, 3), "cores": 1}
 
 
 def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3, keep_outputs=None):
@@ -463,7 +487,51 @@ def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3, keep_outputs=
         out["window_segmentation_128x128"] = time_window_segmentation(fa, torch, dev, calls)
     except Exception as exc:  # noqa: BLE001
         out["window_segmentation_128x128"] = {"error": str(exc)[:200]}
+    for window in (workloads.DECODER_WINDOW, 0):
+        name = f"decoder_{'sliding' if window else 'full'}_16384"
+        try:  # informational, like the segmentation timings
+            out[name] = time_decoder(fa, torch, dev, window, 10, keep_outputs, name)
+        except Exception as exc:  # noqa: BLE001
+            out[name] = {"error": str(exc)[:200]}
     return out
+
+
+def time_decoder(fa, torch, dev, window: int, calls: int, keep_outputs, name: str):
+    """The text decoder's attention (causal, GQA 32/2, head size 128) on one 16384-token
+    sequence: a sliding layer (window 2048) or a full one (window 0); ms per call and
+    TFLOP/s of the attended (query, key) pairs."""
+    T = 16384
+    cu_np = workloads.cu_from_lengths([T])
+    q, k, v = workloads.decoder_qkv(77, T)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    dq, dk, dv = to(q), to(k), to(v)
+    do = torch.empty_like(dq)
+    cu = torch.from_numpy(cu_np.copy()).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(workloads.DECODER_D)
+
+    def call():
+        rc = fa._binding.vt_attn_fwd_swa(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), do.data_ptr(),
+                                         cu.data_ptr(), 1, T, workloads.DECODER_HQ, workloads.DECODER_HKV,
+                                         workloads.DECODER_D, scale, window, stream.cuda_stream)
+        if rc != 0:
+            raise fa.VtAttnError(rc, "vt_attn_fwd_swa")
+    for _ in range(3):
+        call()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(calls):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    fa.check_device_status(stream)
+    ms = e0.elapsed_time(e1) / calls
+    flops = workloads.decoder_flops(cu_np, window)
+    if keep_outputs is not None:
+        keep_outputs[name] = ("decoder", (q, k, v, cu_np, window, scale),
+                              do.float().cpu().numpy().astype(np.float64))
+    return {"dtype": "bf16", "kind": "causal, GQA 32/2, head size 128", "window": window,
+            "tokens": T, "ms": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
 
 
 def time_window_segmentation(fa, torch, dev, calls: int = 20):

@@ -26,7 +26,7 @@ from ._binding import (VT_DTYPE_BF16, VT_DTYPE_F32, VT_OK, VtAttnError, status_s
                        vt_attn_fwd, vt_attn_last_device_status, vt_attn_smem_bytes,
                        vt_attn_validate_seqlens_host, vt_attn_version, vt_attn_workspace_bytes)
 
-__all__ = ["attn_fwd", "attn_fwd_host", "window_partition", "permute_rows", "check_permute_rows",
+__all__ = ["attn_fwd", "attn_fwd_swa", "attn_fwd_host", "window_partition", "permute_rows", "check_permute_rows",
            "rope2d", "attn_fwd_rope2d",
            "check_device_status", "VtAttnError", "vt_attn_fwd",
            "vt_attn_validate_seqlens_host", "vt_attn_smem_bytes", "vt_attn_workspace_bytes",
@@ -80,6 +80,47 @@ def attn_fwd(q, k, v, cu_seqlens, scale: float | None = None, out=None, stream=N
                          code, handle)
     if rc != VT_OK:
         raise VtAttnError(rc, "vt_attn_fwd")
+    return out
+
+
+def attn_fwd_swa(q, k, v, cu_seqlens, window: int = 0, scale: float | None = None, out=None,
+                 stream=None):
+    """The text decoder's attention: causal over packed segments, query token i attending
+    keys j <= i of its segment (and j > i - window when window > 0), query head h reading
+    key/value head h // (Hq // Hkv).
+
+    q: bfloat16 CUDA tensor [T, Hq, 128]; k, v: [T, Hkv, 128]; cu_seqlens: int32 CUDA tensor
+    [num_segments + 1].  scale: default 1/sqrt(128).  Returns ``out`` ([T, Hq, 128]).
+    """
+    import torch
+    if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape or k.shape[0] != q.shape[0] \
+            or k.shape[2] != q.shape[2]:
+        raise ValueError(f"attn_fwd_swa: q [T, Hq, D], k and v [T, Hkv, D] expected, got "
+                         f"{tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens", cu_seqlens)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"attn_fwd_swa: {name} must be a contiguous CUDA tensor")
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("attn_fwd_swa: q, k, v must be bfloat16")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+        raise TypeError("attn_fwd_swa: cu_seqlens must be a 1-D int32 tensor")
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("attn_fwd_swa: out must be a contiguous tensor like q")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(q.device):
+        rc = _binding.vt_attn_fwd_swa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      cu_seqlens.data_ptr(), cu_seqlens.numel() - 1, T, Hq, Hkv, D,
+                                      float(scale), int(window), handle)
+    if rc != VT_OK:
+        raise VtAttnError(rc, "vt_attn_fwd_swa")
     return out
 
 

@@ -39,6 +39,7 @@ EXPORTED = (
     "vt_permute_rows_check",
     "vt_rope2d",
     "vt_attn_fwd_rope2d",
+    "vt_attn_fwd_swa",
     "vt_attn_status_string",
     "vt_attn_version",
 )
@@ -80,6 +81,8 @@ def _load():
     lib.vt_permute_rows.restype = ctypes.c_int
     lib.vt_attn_fwd_rope2d.argtypes = [P, P, P, P, P, I32, I32, I32, I32, F, P, F, P, P]
     lib.vt_attn_fwd_rope2d.restype = ctypes.c_int
+    lib.vt_attn_fwd_swa.argtypes = [P, P, P, P, P, I32, I32, I32, I32, I32, F, I32, P]
+    lib.vt_attn_fwd_swa.restype = ctypes.c_int
     lib.vt_rope2d.argtypes = [P, P, P, I32, I32, I32, F, P]
     lib.vt_rope2d.restype = ctypes.c_int
     lib.vt_permute_rows_check.argtypes = [P]
@@ -167,6 +170,14 @@ def vt_attn_fwd_rope2d(q: int, k: int, v: int, out: int, cu_seqlens: int, num_se
     """Attention over rope(Q), rope(K) (bf16): Q rotated in the kernel, K into k_rot."""
     return lib.vt_attn_fwd_rope2d(q, k, v, out, cu_seqlens, num_segments, total_tokens, H, D,
                                   ctypes.c_float(scale), pos, ctypes.c_float(theta), k_rot, stream)
+
+
+def vt_attn_fwd_swa(q: int, k: int, v: int, out: int, cu_seqlens: int, num_segments: int,
+                    total_tokens: int, Hq: int, Hkv: int, D: int, scale: float, window: int,
+                    stream: int) -> int:
+    """Causal attention with a local window (0: none) and grouped-query heads (bf16, D 128)."""
+    return lib.vt_attn_fwd_swa(q, k, v, out, cu_seqlens, num_segments, total_tokens, Hq, Hkv, D,
+                               ctypes.c_float(scale), window, stream)
 
 
 def vt_permute_rows_check(stream: int) -> int:

@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libvtattn.so")
 
 SOURCES = ["vt_attn.cu", "vt_attn_noalloc.cu", "sched.cu", "attn_bf16_sm100.cu", "attn_f32split_sm100.cu",
-           "window.cu", "rope2d.cu"]
+           "window.cu", "rope2d.cu", "attn_swa_bf16_sm100.cu"]
 HEADERS = ["ptx.cuh", "internal.h", "rope2d.cuh"]
 
 NVCC_FLAGS = [

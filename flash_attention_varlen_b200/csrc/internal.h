@@ -112,6 +112,23 @@ size_t f32_smem_bytes();
 cudaError_t prepare_attn_f32();  // opt in to the kernel's dynamic shared memory (per device)
 cudaError_t launch_attn_f32(const F32Args& args, int grid, cudaStream_t stream);
 
+// Text decoder attention: causal, a local window (0: none), grouped-query heads; bf16,
+// head size 128.  Units are 128 query rows of one (segment, query head).
+constexpr int kSwaBlockRows = 128;
+constexpr int kSwaHeadDim = 128;
+struct SwaArgs {
+  void* out;
+  const WorkHeader* hdr;
+  const WorkEntry* entries;
+  int* dev_status;
+  int32_t Hq, Hkv, window;
+  float scale_log2;  // scale * log2(e), signed
+};
+size_t swa_smem_bytes();
+cudaError_t prepare_attn_swa();  // opt in to the kernel's dynamic shared memory (per device)
+cudaError_t launch_attn_swa(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const SwaArgs& args, int grid, cudaStream_t stream);
+
 // ---------------------------------------------------------------- host launcher
 // One forward call as the entry points receive it (validated by check_fwd_args).
 struct FwdCall {

@@ -29,6 +29,7 @@ struct DeviceInfo {
   int num_sms = 0;
   bool bf16_ready = false;
   bool f32_ready = false;
+  bool swa_ready = false;
 };
 
 struct Scratch {
@@ -62,15 +63,16 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-// [T, H, 96] bf16 viewed as (d, h, t); a box is 32 columns x 1 head x 128 rows, stored
+// [T, H, D] bf16 viewed as (d, h, t); a box is 32 columns x 1 head x 128 rows, stored
 // with the 64-byte swizzle (32 columns = 64 bytes per row) the MMA descriptors expect.
-vt_status make_tensor_map(CUtensorMap* map, const void* base, int32_t T, int32_t H) {
+vt_status make_tensor_map(CUtensorMap* map, const void* base, int32_t T, int32_t H,
+                          int32_t D = kHeadDim) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return VT_ERR_CUDA;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(H),
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(T)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2,
-                                 static_cast<cuuint64_t>(H) * kHeadDim * 2};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(H) * D * 2};
   const cuuint32_t box[3] = {32, 1, 128};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
@@ -276,6 +278,53 @@ vt_status fwd_impl(const vt::FwdCall& c) {
       vt::launch_fwd(c, hdr, reinterpret_cast<vt::WorkEntry*>(hdr + 1), slot));
 }
 
+// The text decoder's attention: validated arguments, the prepass (128-row entries) and the
+// kernel, on the stream's scratch.
+vt_status swa_impl(const void* q, const void* k, const void* v, void* out, const int32_t* cu,
+                   int32_t n, int32_t T, int32_t Hq, int32_t Hkv, float scale, int32_t window,
+                   cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VT_ERR_CUDA;
+  DeviceInfo* di = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    vt_status st = device_info(dev, &di);
+    if (st != VT_OK) return st;
+    if (!di->swa_ready) {
+      if (vt::prepare_attn_swa() != cudaSuccess) return VT_ERR_CUDA;
+      di->swa_ready = true;
+    }
+  }
+  CUtensorMap tq, tk, tv;
+  vt_status st;
+  if ((st = make_tensor_map(&tq, q, T, Hq, vt::kSwaHeadDim)) != VT_OK) return st;
+  if ((st = make_tensor_map(&tk, k, T, Hkv, vt::kSwaHeadDim)) != VT_OK) return st;
+  if ((st = make_tensor_map(&tv, v, T, Hkv, vt::kSwaHeadDim)) != VT_OK) return st;
+  std::lock_guard<std::mutex> lock(g_mu);
+  Scratch* sc = nullptr;
+  st = scratch_for(dev, stream, vt::scratch_bytes_for(T, n, vt::kSwaBlockRows), &sc);
+  if (st != VT_OK) return st;
+  auto* hdr = static_cast<vt::WorkHeader*>(sc->ptr);
+  auto* entries = reinterpret_cast<vt::WorkEntry*>(hdr + 1);
+  const int slot = static_cast<int>(sc->calls++ & 1u);
+  sc->last_slot = slot;
+  if (vt::launch_schedule(cu, n, T, vt::kSwaBlockRows, slot, hdr, entries, stream) != cudaSuccess)
+    return VT_ERR_CUDA;
+  vt::SwaArgs a;
+  a.out = out;
+  a.hdr = hdr;
+  a.entries = entries;
+  a.dev_status = &hdr->status[slot];
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.window = window;
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  const long long units = vt::max_work_entries(T, n, vt::kSwaBlockRows) * static_cast<long long>(Hq);
+  const long long cap = 2ll * di->num_sms;  // two CTAs per SM
+  const int grid = static_cast<int>(units < cap ? units : cap);
+  return vt::launch_attn_swa(tq, tk, tv, a, grid, stream) == cudaSuccess ? VT_OK : VT_ERR_CUDA;
+}
+
 vt::FwdCall make_call(const void* q, const void* k, const void* v, void* out,
                       const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
                       int32_t H, float scale, vt_dtype dtype, void* stream_ptr, int32_t stall) {
@@ -432,6 +481,32 @@ vt_status vt_attn_fwd_rope2d(const void* q, const void* k, const void* v, void* 
   c.rope_pos = pos;
   c.rope_theta = theta;
   return fwd_impl(c);
+}
+
+vt_status vt_attn_fwd_swa(const void* q, const void* k, const void* v, void* out,
+                          const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                          int32_t Hq, int32_t Hkv, int32_t D, float scale, int32_t window,
+                          void* stream_ptr) {
+  if (Hq < 1 || Hkv < 1 || D < 1 || num_segments < 0 || total_tokens < 0 || window < 0)
+    return VT_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || !std::isfinite(scale)) return VT_ERR_INVALID_ARG;
+  if (D != vt::kSwaHeadDim) return VT_ERR_UNSUPPORTED;
+  if (num_segments == 0) return total_tokens == 0 ? VT_OK : VT_ERR_BAD_SEQLENS;
+  if (!cu_seqlens) return VT_ERR_NULL;
+  if (total_tokens == 0) return VT_OK;
+  if (!q || !k || !v || !out) return VT_ERR_NULL;
+  const uintptr_t align_or = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                             reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+  if (align_or & 15u) return VT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) return VT_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(Hq) * D > (1 << 20)) return VT_ERR_INVALID_ARG;
+  const size_t qbytes = static_cast<size_t>(total_tokens) * Hq * D * 2;
+  const size_t kvbytes = static_cast<size_t>(total_tokens) * Hkv * D * 2;
+  if (ranges_overlap(out, qbytes, q, qbytes) || ranges_overlap(out, qbytes, k, kvbytes) ||
+      ranges_overlap(out, qbytes, v, kvbytes))
+    return VT_ERR_INVALID_ARG;
+  return swa_impl(q, k, v, out, cu_seqlens, num_segments, total_tokens, Hq, Hkv, scale, window,
+                  static_cast<cudaStream_t>(stream_ptr));
 }
 
 vt_status vt_rope2d(const void* x, void* out, const int32_t* pos, int32_t total_tokens, int32_t H,

@@ -268,6 +268,32 @@ vt_status vt_attn_fwd_rope2d(const void* q, const void* k, const void* v, void* 
                              int32_t H, int32_t D, float scale, const int32_t* pos, float theta,
                              void* k_rot, void* stream);
 
+/*
+ * The text decoder's attention (the Muse Glimmer next-steps document, "Architecture / Text
+ * decoder": 32 query heads over 2 key/value heads, head size 128, a local window of 2048
+ * tokens on the sliding layers): causal attention with an optional local window and
+ * grouped-query heads, over packed segments.  For query token i of segment s and query
+ * head h:
+ *     O[i,h,:] = sum_j softmax_j(scale * <Q[i,h,:], K[j,g,:]>) V[j,g,:],
+ *     j over the tokens of s with j <= i, and j > i - window when window > 0,
+ *     g = h / (Hq / Hkv).
+ *   q, out        device pointers, bf16 [total_tokens, Hq, D] row-major, 16-byte aligned.
+ *   k, v          device pointers, bf16 [total_tokens, Hkv, D] row-major, 16-byte aligned.
+ *   cu_seqlens    device pointer, int32 [num_segments + 1], validated on the device as for
+ *                 vt_attn_fwd (a malformed one is reported by vt_attn_last_device_status).
+ *   Hq, Hkv       Hq a multiple of Hkv (Hq == Hkv: ordinary multi-head attention).
+ *   D             only 128 (VT_ERR_UNSUPPORTED otherwise).
+ *   scale         any finite float (the decoder folds its query multiplier into it).
+ *   window        >= 0; 0 means no window (a full-attention layer).
+ * out must not overlap q, k or v.  bf16 in and out, f32 accumulation.  Asynchronous on
+ * `stream`; the library's per-stream scratch is shared with vt_attn_fwd.  Returns as
+ * vt_attn_fwd.
+ */
+vt_status vt_attn_fwd_swa(const void* q, const void* k, const void* v, void* out,
+                          const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,
+                          int32_t Hq, int32_t Hkv, int32_t D, float scale, int32_t window,
+                          void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* vt_attn_status_string(vt_status status);
 
