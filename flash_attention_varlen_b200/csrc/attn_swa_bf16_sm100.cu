@@ -45,7 +45,7 @@ struct Smem {
   uint8_t k[kTileBytes];
   uint8_t v[kTileBytes];
   uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty;
-  uint64_t s_full, p_full, o_done, drain;
+  uint64_t s_full, p_full[2], o_done, drain;  // p_full: one per 64-key half of P
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&sm.v_full, 1);
     mbar_init(&sm.v_empty, 1);
     mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.p_full, 128);
+    mbar_init(&sm.p_full[0], 128);
+    mbar_init(&sm.p_full[1], 128);
     mbar_init(&sm.o_done, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -204,13 +205,18 @@ __global__ void __launch_bounds__(kThreads, 2)
           mma_commit(&sm.s_full);
           mma_commit(&sm.k_empty);
           if (j + 1 == x.nkv) mma_commit(&sm.q_empty);
-          if (!mbar_wait_bounded(&sm.p_full, t & 1, abort_flag, dev_status)) { ok = false; break; }
           if (!mbar_wait_bounded(&sm.v_full, t & 1, abort_flag, dev_status)) { ok = false; break; }
-          tc_fence_after();
+          // PV on each 64-key half of P as soon as the softmax has stored it
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tmem + kColO, tmem + kColS + kk * 8, dv + static_cast<uint64_t>((kk * 1024) >> 4),
-                   idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int half = 0; half < 2; ++half) {
+            if (!mbar_wait_bounded(&sm.p_full[half], t & 1, abort_flag, dev_status)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = half * 4; kk < half * 4 + 4; ++kk)
+              mma_ts(tmem + kColO, tmem + kColS + kk * 8, dv + static_cast<uint64_t>((kk * 1024) >> 4),
+                     idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (!ok) break;
           mma_commit(&sm.o_done);
           mma_commit(&sm.v_empty);
         }
@@ -240,6 +246,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         // valid key columns [ka, kb) of this tile for this row
         const int ka = row_in ? max(lo_i - kv0, 0) : kBN;
         const int kb = row_in ? min(i - kv0 + 1, kBN) : 0;
+        // tiles inside every row's allowed range (most of a window) skip the masking
+        const bool need_mask = __any_sync(0xffffffffu, ka > 0 || kb < kBN);
         float pm[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
@@ -251,10 +259,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_ld32(tS + half * 64 + 32, su + 32);
           tmem_ld_wait();
           reg_fence<64>(su);
+          if (need_mask) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const int col = half * 64 + e;
-            if (col < ka || col >= kb) sf[e] = -INFINITY;
+            for (int e = 0; e < 64; ++e) {
+              const int col = half * 64 + e;
+              if (col < ka || col >= kb) sf[e] = -INFINITY;
+            }
           }
 #pragma unroll
           for (int e = 0; e < 64; e += 16) {
@@ -302,21 +312,31 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_ld_wait();
           reg_fence<64>(su);
           uint32_t p[32];
+          float2 l2 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int e2 = 0; e2 < 32; ++e2) {
-            const int col = half * 64 + 2 * e2;
             const float2 tt = ffma2(make_float2(sf[2 * e2], sf[2 * e2 + 1]), c2, nm2);
-            const float p0 = (live && col >= ka && col < kb) ? ex2_approx(tt.x) : 0.f;
-            const float p1 = (live && col + 1 >= ka && col + 1 < kb) ? ex2_approx(tt.y) : 0.f;
-            p[e2] = pack_bf16x2(p0, p1);
+            float2 pe;
+            if (e2 % 3 == 2) {
+              pe = exp2_poly2(tt);  // a third on the FMA pipe, as the vision kernel
+            } else {
+              pe = make_float2(ex2_approx(tt.x), ex2_approx(tt.y));
+            }
+            if (need_mask) {
+              const int col = half * 64 + 2 * e2;
+              if (!live || col < ka || col >= kb) pe.x = 0.f;
+              if (!live || col + 1 < ka || col + 1 >= kb) pe.y = 0.f;
+            }
+            p[e2] = pack_bf16x2(pe.x, pe.y);
             // the row sum of the rounded weights the PV product uses
-            l += __uint_as_float(p[e2] << 16) + __uint_as_float(p[e2] & 0xFFFF0000u);
+            l2 = fadd2(l2, make_float2(__uint_as_float(p[e2] << 16), __uint_as_float(p[e2] & 0xFFFF0000u)));
           }
+          l += l2.x + l2.y;
           tmem_st32(tS + half * 32, p);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&sm.p_full[half]);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&sm.p_full);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 -> HBM
