@@ -57,7 +57,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time budget of the oracle sample")
-    ap.add_argument("--single-layer", choices=["full", "window", "varlen8"], default=None,
+    ap.add_argument("--single-layer", choices=["full", "window", "varlen8", "f32_4096",
+                                               "decoder_sliding", "decoder_full"], default=None,
                     help="profiling aid: run only one layer (full = 1 x 16384 tok, window = "
                          "16 x 1024 tok, varlen8 = eight images of unequal size) warmup + "
                          "steps times and print its timing")
@@ -661,32 +662,49 @@ def run_reference(args):
 
 
 def run_single_layer(args):
-    """One layer type of the tower, called warmup + steps times (for ncu captures)."""
+    """One layer, called warmup + steps times (for ncu captures): a tower layer type, the
+    eight-image batch, a 4096-token f32 segment (the f32 arm) or the text decoder's sliding
+    or full layer on a 16384-token sequence."""
     import torch
     import flash_attention_varlen_b200 as fa
-    if args.single_layer == "varlen8":  # eight images of unequal size (the scheduler's case)
-        case = workloads.varlen8_case(0)
-    else:
-        case = workloads.tower_layer_case(3 if args.single_layer == "full" else 0, GRID)
-    q, k, v = case.inputs()
     dev = torch.device("cuda", 0)
-    to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
-    dq, dk, dv = to(q), to(k), to(v)
-    out = torch.empty_like(dq)
-    cu = torch.from_numpy(case.cu_seqlens.copy()).to(dev)
+    bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    if args.single_layer.startswith("decoder_"):
+        window = workloads.DECODER_WINDOW if args.single_layer == "decoder_sliding" else 0
+        cu_np = workloads.cu_from_lengths([GRID * GRID])
+        q, k, v = workloads.decoder_qkv(77, GRID * GRID)
+        dq, dk, dv = bf16(q), bf16(k), bf16(v)
+        flops = workloads.decoder_flops(cu_np, window)
+        cu = torch.from_numpy(cu_np.copy()).to(dev)
+        out = torch.empty_like(dq)
+        call = lambda: fa.attn_fwd_swa(dq, dk, dv, cu, window=window, out=out)
+    else:
+        if args.single_layer == "varlen8":  # eight images of unequal size (the scheduler's case)
+            case = workloads.varlen8_case(0)
+        elif args.single_layer == "f32_4096":
+            case = workloads.Case("f32_4096", workloads.cu_from_lengths([4096]), seed=5, dtype="f32")
+        else:
+            case = workloads.tower_layer_case(3 if args.single_layer == "full" else 0, GRID)
+        q, k, v = case.inputs()
+        to = bf16 if case.dtype == "bf16" else (lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev))
+        dq, dk, dv = to(q), to(k), to(v)
+        flops = case.flops()
+        cu = torch.from_numpy(case.cu_seqlens.copy()).to(dev)
+        out = torch.empty_like(dq)
+        call = lambda: fa.attn_fwd(dq, dk, dv, cu, scale=SCALE, out=out)
     for _ in range(args.warmup):
-        fa.attn_fwd(dq, dk, dv, cu, scale=SCALE, out=out)
+        call()
     fa.check_device_status()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        fa.attn_fwd(dq, dk, dv, cu, scale=SCALE, out=out)
+        call()
     e1.record()
     torch.cuda.synchronize()
     fa.check_device_status()
     ms = e0.elapsed_time(e1) / max(1, args.steps)
     print(json.dumps({"single_layer": args.single_layer, "ms_per_call": round(ms, 4),
-                      "tflops": round(case.flops() / (ms * 1e-3) / 1e12, 2),
+                      "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
                       "calls": args.steps, "note": "back-to-back calls on one layer's inputs"}))
 
 
