@@ -7,45 +7,58 @@
 // window); query head h reads key/value head h / (Hq / Hkv).  Flash-style with a running
 // softmax, as the vision kernel: scores never leave the SM.
 //
-// One CTA works through units of 128 query rows of one (segment, query head); two CTAs
-// share an SM (96 KB of shared memory and 256 TMEM columns each), so one CTA's tensor work
-// runs while the other is in its softmax.  A unit visits only the key tiles its rows can
-// see: from the window start of its first row to its last row.
+// One CTA per SM works through units of 256 query rows of one (segment, query head): two
+// 128-row Q tiles that share every K/V tile, as in the vision kernel, so the tensor core
+// works on one tile while the other is in its softmax.  A unit visits only the key tiles its
+// rows can see (from the window start of its first row to its last row); a tile that one Q
+// tile cannot see at all costs that tile's MMAs and a masked softmax pass.
 //
-//   warp 4 (loader)  : TMA loads of the Q tile and of each K and V tile (single buffers,
-//                      64-byte swizzle, four 32-column chunks).
-//   warp 5 (MMA)     : S = Q K^T (SS, M128 N128 K128), then O (+)= P V (TS, P from TMEM).
-//   warps 0-3        : softmax, one thread per query row: the row's allowed keys of the
-//                      tile, row max with a deferred rescale, p = 2^(s c - m) packed to
-//                      bf16 over S in TMEM, the row sum of the rounded p in f32; the
-//                      epilogue O / l -> bf16 -> HBM.
+//   warp 8 (loader)  : TMA loads of the two Q tiles and of each K and V tile into 2-stage
+//                      rings (64-byte swizzle, four 32-column chunks).
+//   warp 9 (MMA)     : one thread issues S_i = Q_i K^T (SS, M128 N128 K128) and
+//                      O_i (+)= P_i V (TS, P from TMEM, N128) in the order
+//                      S0 S1 | PV0 S0' | PV1 S1' | ...
+//   warps 0-3, 4-7   : softmax for Q tiles 0 and 1, one thread per query row: the row's
+//                      allowed keys of the tile, row max with a deferred rescale,
+//                      p = 2^(s c - m) packed to bf16 over S in TMEM (in two 64-key halves,
+//                      each handed to the PV as soon as it is stored), the row sum of the
+//                      rounded p in f32; the epilogue O / l -> bf16 -> HBM.
 //
-// TMEM (256 columns): S [0,128) (P overlays its first 64 columns), O [128,256).
-// Every mbarrier wait is bounded and an abort flag lets all roles leave together.
+// TMEM (512 columns): S0 [0,128), O0 [128,256), S1 [256,384), O1 [384,512); P_i overlays
+// the first 64 columns of S_i.  Every mbarrier wait is bounded and an abort flag lets all
+// roles leave together.
+#include <type_traits>
+
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace vt {
 namespace {
 
-constexpr int kBM = kSwaBlockRows;  // 128 query rows per unit
+constexpr int kBM = 128;            // query rows per Q tile
+constexpr int kUnitRows = kSwaBlockRows;  // 256: two Q tiles per unit
 constexpr int kBN = 128;            // keys per tile
 constexpr int kD = 128;
 constexpr int kChunks = kD / 32;              // 32-column (64-byte) chunks per row
 constexpr int kChunkBytes = 128 * 64;         // 128 rows x 32 bf16
 constexpr int kTileBytes = kChunks * kChunkBytes;  // 32 KB
-constexpr int kThreads = 192;
-constexpr int kWarpLoad = 4, kWarpMma = 5;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColO = 128;
+constexpr int kStages = 2;                    // K and V ring depth
+constexpr int kThreads = 320;
+constexpr int kWarpLoad = 8, kWarpMma = 9;
+constexpr uint32_t kTmemCols = 512;
+// TMEM columns of Q tile i: S_i at 256 i, O_i at 256 i + 128
+__host__ __device__ constexpr uint32_t col_s(int tile) { return 256u * tile; }
+__host__ __device__ constexpr uint32_t col_o(int tile) { return 256u * tile + 128u; }
 constexpr float kRescaleThreshold = 3.0f;  // log2 units, as the vision kernel
 
 struct Smem {
-  uint8_t q[kTileBytes];
-  uint8_t k[kTileBytes];
-  uint8_t v[kTileBytes];
-  uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty;
-  uint64_t s_full, p_full[2], o_done, drain;  // p_full: one per 64-key half of P
+  uint8_t q[2][kTileBytes];
+  uint8_t k[kStages][kTileBytes];
+  uint8_t v[kStages][kTileBytes];
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2][2], o_done[2];  // per Q tile (p_full: per 64-key half)
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -54,6 +67,7 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 struct Unit {
   int head, kv_head, q0, seg_start, seg_end;
   int j0, nkv;  // first key tile (from the segment start) and the tile count
+  bool has_q1;  // the second Q tile holds rows of the segment
 };
 
 // This CTA's units: a snake over the CTAs, entry-major with the query heads inner (the
@@ -71,9 +85,10 @@ struct Units {
     x->kv_head = x->head / group;
     x->seg_start = we.seg_start;
     x->seg_end = we.seg_end;
-    const int nblocks = (we.seg_end - we.seg_start + kBM - 1) / kBM;
-    x->q0 = we.seg_start + (nblocks - 1 - we.qblock) * kBM;
-    const int q_last = min(x->q0 + kBM, we.seg_end) - 1;
+    const int nblocks = (we.seg_end - we.seg_start + kUnitRows - 1) / kUnitRows;
+    x->q0 = we.seg_start + (nblocks - 1 - we.qblock) * kUnitRows;
+    x->has_q1 = x->q0 + kBM < we.seg_end;
+    const int q_last = min(x->q0 + kUnitRows, we.seg_end) - 1;
     const int lo = window > 0 ? max(we.seg_start, x->q0 - window + 1) : we.seg_start;
     x->j0 = (lo - we.seg_start) / kBN;
     x->nkv = (q_last - we.seg_start) / kBN - x->j0 + 1;
@@ -100,7 +115,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_swa_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ SwaArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -111,14 +126,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
-    mbar_init(&sm.k_full, 1);
-    mbar_init(&sm.k_empty, 1);
-    mbar_init(&sm.v_full, 1);
-    mbar_init(&sm.v_empty, 1);
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.p_full[0], 128);
-    mbar_init(&sm.p_full[1], 128);
-    mbar_init(&sm.o_done, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i][0], 128);
+      mbar_init(&sm.p_full[i][1], 128);
+      mbar_init(&sm.o_done[i], 1);
+    }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -157,90 +176,146 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == kWarpLoad) {
     // ------------------------------------------------------------ loader
     if (lane == 0) {
-      uint32_t nk = 0, nv = 0, n = 0;  // K tiles, V tiles and Q tiles issued
+      uint32_t nq = 0, nk = 0, nv = 0;  // Q pairs, K tiles and V tiles issued
       Unit x;
       bool ok = true;
       for (long long k = 0; ok && us.get(k, &x); ++k) {
-        if (n > 0 && !mbar_wait_bounded(&sm.q_empty, (n - 1) & 1, abort_flag, dev_status)) break;
-        mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-        tma_tile(sm.q, &tq, &sm.q_full, x.head, x.q0);
-        ++n;
+        if (nq > 0 && !mbar_wait_bounded(&sm.q_empty, (nq - 1) & 1, abort_flag, dev_status)) break;
+        mbar_arrive_expect_tx(&sm.q_full, x.has_q1 ? 2 * kTileBytes : kTileBytes);
+        tma_tile(sm.q[0], &tq, &sm.q_full, x.head, x.q0);
+        if (x.has_q1) tma_tile(sm.q[1], &tq, &sm.q_full, x.head, x.q0 + kBM);
+        ++nq;
         for (int j = 0; j < x.nkv; ++j) {
           const int row0 = x.seg_start + (x.j0 + j) * kBN;
-          if (nk > 0 && !mbar_wait_bounded(&sm.k_empty, (nk - 1) & 1, abort_flag, dev_status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sm.k_full, kTileBytes);
-          tma_tile(sm.k, &tk, &sm.k_full, x.kv_head, row0);
+          const uint32_t sk = nk % kStages, sv = nv % kStages;
+          if (nk >= kStages &&
+              !mbar_wait_bounded(&sm.k_empty[sk], (nk / kStages - 1) & 1, abort_flag, dev_status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.k_full[sk], kTileBytes);
+          tma_tile(sm.k[sk], &tk, &sm.k_full[sk], x.kv_head, row0);
           ++nk;
-          if (nv > 0 && !mbar_wait_bounded(&sm.v_empty, (nv - 1) & 1, abort_flag, dev_status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sm.v_full, kTileBytes);
-          tma_tile(sm.v, &tv, &sm.v_full, x.kv_head, row0);
+          if (nv >= kStages &&
+              !mbar_wait_bounded(&sm.v_empty[sv], (nv / kStages - 1) & 1, abort_flag, dev_status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.v_full[sv], kTileBytes);
+          tma_tile(sm.v[sv], &tv, &sm.v_full[sv], x.kv_head, row0);
           ++nv;
         }
       }
-      // every copy issued lands before the CTA exits, aborted or not
-      if (n > 0) mbar_wait_drain(&sm.q_full, (n - 1) & 1);
-      if (nk > 0) mbar_wait_drain(&sm.k_full, (nk - 1) & 1);
-      if (nv > 0) mbar_wait_drain(&sm.v_full, (nv - 1) & 1);
+      // every copy issued lands before the CTA exits, aborted or not: the last use of each
+      // ring stage
+      if (nq > 0) mbar_wait_drain(&sm.q_full, (nq - 1) & 1);
+      for (uint32_t s = 0; s < kStages; ++s) {
+        if (nk > s) mbar_wait_drain(&sm.k_full[s], ((nk - 1 - s) / kStages) & 1);
+        if (nv > s) mbar_wait_drain(&sm.v_full[s], ((nv - 1 - s) / kStages) & 1);
+      }
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = make_idesc_bf16(kBM, kBN, false, false, a.scale_log2 < 0.0f);
       const uint32_t idesc_pv = make_idesc_bf16(kBM, kD, false, true, false);
-      const uint64_t dq = qk_desc(smem_u32(sm.q)), dk = qk_desc(smem_u32(sm.k));
-      const uint64_t dv = pv_desc(smem_u32(sm.v));
-      uint32_t t = 0, n = 0;
-      Unit x;
-      bool ok = true;
-      for (long long k = 0; ok && us.get(k, &x); ++k, ++n) {
-        if (!mbar_wait_bounded(&sm.q_full, n & 1, abort_flag, dev_status)) break;
-        for (int j = 0; j < x.nkv; ++j, ++t) {
-          if (!mbar_wait_bounded(&sm.k_full, t & 1, abort_flag, dev_status)) { ok = false; break; }
+      // descriptors: Q tile i starts i * kTileBytes after q[0]; ring stage s of K (V) starts
+      // s * kTileBytes after k[0] (v[0])
+      const uint64_t dq0 = qk_desc(smem_u32(sm.q[0])), dk0 = qk_desc(smem_u32(sm.k[0]));
+      const uint64_t dv0 = pv_desc(smem_u32(sm.v[0]));
+      constexpr uint64_t kTileStep = kTileBytes >> 4;
+      auto issue_qk = [&](auto tile_c, uint32_t st) {
+        constexpr int tile = decltype(tile_c)::value;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 1) * kChunkBytes + (kk & 1) * 32) >> 4);
+          mma_ss(tmem + col_s(tile), dq0 + tile * kTileStep + off, dk0 + st * kTileStep + off, idesc_qk,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sm.s_full[tile]);
+      };
+      uint32_t nq = 0, kc = 0, vc = 0, pc0 = 0, pc1 = 0;
+      // O_i (+)= P_i V for one key tile, each 64-key half as soon as the softmax stored it
+      auto issue_pv = [&](auto tile_c, uint32_t sv, bool accumulate) {
+        constexpr int tile = decltype(tile_c)::value;
+        uint32_t& pc = tile == 0 ? pc0 : pc1;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait_bounded(&sm.p_full[tile][half], pc & 1, abort_flag, dev_status)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(((kk >> 1) * kChunkBytes + (kk & 1) * 32) >> 4);
-            mma_ss(tmem + kColS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&sm.s_full);
-          mma_commit(&sm.k_empty);
-          if (j + 1 == x.nkv) mma_commit(&sm.q_empty);
-          if (!mbar_wait_bounded(&sm.v_full, t & 1, abort_flag, dev_status)) { ok = false; break; }
-          // PV on each 64-key half of P as soon as the softmax has stored it
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            if (!mbar_wait_bounded(&sm.p_full[half], t & 1, abort_flag, dev_status)) { ok = false; break; }
+          for (int kk = half * 4; kk < half * 4 + 4; ++kk)
+            mma_ts(tmem + col_o(tile), tmem + col_s(tile) + kk * 8,
+                   dv0 + sv * kTileStep + static_cast<uint64_t>((kk * 1024) >> 4), idesc_pv,
+                   (accumulate || kk > 0) ? 1u : 0u);
+        }
+        ++pc;
+        mma_commit(&sm.o_done[tile]);
+        return true;
+      };
+      using T0 = std::integral_constant<int, 0>;
+      using T1 = std::integral_constant<int, 1>;
+      Unit x;
+      bool ok = true;
+      for (long long k = 0; ok && us.get(k, &x); ++k, ++nq) {
+        if (!mbar_wait_bounded(&sm.q_full, nq & 1, abort_flag, dev_status)) break;
+        {
+          const uint32_t st = kc % kStages;
+          if (!mbar_wait_bounded(&sm.k_full[st], (kc / kStages) & 1, abort_flag, dev_status)) break;
+          tc_fence_after();
+          issue_qk(T0{}, st);
+          if (x.has_q1) issue_qk(T1{}, st);
+          mma_commit(&sm.k_empty[st]);
+          ++kc;
+          if (x.nkv == 1) mma_commit(&sm.q_empty);
+        }
+        for (int j = 0; j < x.nkv; ++j, ++vc) {
+          const uint32_t sv = vc % kStages;
+          const bool more = j + 1 < x.nkv;
+          if (!mbar_wait_bounded(&sm.v_full[sv], (vc / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
+          if (!issue_pv(T0{}, sv, j > 0)) { ok = false; break; }
+          if (!x.has_q1) mma_commit(&sm.v_empty[sv]);
+          const uint32_t st = kc % kStages;
+          if (more) {
+            if (!mbar_wait_bounded(&sm.k_full[st], (kc / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int kk = half * 4; kk < half * 4 + 4; ++kk)
-              mma_ts(tmem + kColO, tmem + kColS + kk * 8, dv + static_cast<uint64_t>((kk * 1024) >> 4),
-                     idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            issue_qk(T0{}, st);
           }
-          if (!ok) break;
-          mma_commit(&sm.o_done);
-          mma_commit(&sm.v_empty);
+          if (x.has_q1) {
+            if (!issue_pv(T1{}, sv, j > 0)) { ok = false; break; }
+            mma_commit(&sm.v_empty[sv]);
+          }
+          if (more) {
+            if (x.has_q1) issue_qk(T1{}, st);
+            mma_commit(&sm.k_empty[st]);
+            ++kc;
+            if (j + 2 == x.nkv) mma_commit(&sm.q_empty);
+          }
         }
       }
       mma_commit(&sm.drain);
       mbar_wait_drain(&sm.drain, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax
-    const int r = tid;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kColS, tO = tmem + lane_base + kColO;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;
+    const int r = tid & 127;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + col_s(wg), tO = tmem + lane_base + col_o(wg);
     const float c = fabsf(a.scale_log2);  // the sign of scale is in the QK descriptor
-    uint32_t t = 0;
+    uint32_t s_cnt = 0, o_base = 0;
     Unit x;
     for (long long k = 0; us.get(k, &x); ++k) {
+      if (wg == 1 && !x.has_q1) continue;
       bool ok = true;
-      const int i = x.q0 + r;  // this thread's query row (token)
+      const int i = x.q0 + wg * kBM + r;  // this thread's query row (token)
       const bool row_in = i < x.seg_end;
       // allowed keys of row i: [lo_i, i]; none for rows past the segment end
       const int lo_i = a.window > 0 ? max(x.seg_start, i - a.window + 1) : x.seg_start;
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < x.nkv; ++j, ++t) {
-        if (!warp_wait(&sm.s_full, t & 1, abort_flag, dev_status)) { ok = false; break; }
+      for (int j = 0; j < x.nkv; ++j) {
+        if (!warp_wait(&sm.s_full[wg], s_cnt & 1, abort_flag, dev_status)) { ok = false; break; }
+        ++s_cnt;
         tc_fence_after();
         const int kv0 = x.seg_start + (x.j0 + j) * kBN;
         // valid key columns [ka, kb) of this tile for this row
@@ -335,12 +410,13 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_st32(tS + half * 32, p);
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&sm.p_full[half]);
+          mbar_arrive(&sm.p_full[wg][half]);
         }
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 -> HBM
-      if (!warp_wait(&sm.o_done, (t - 1) & 1, abort_flag, dev_status)) break;
+      if (!warp_wait(&sm.o_done[wg], (o_base + x.nkv - 1) & 1, abort_flag, dev_status)) break;
+      o_base += x.nkv;
       tc_fence_after();
       const float inv_l = 1.0f / l;
       uint8_t* row = static_cast<uint8_t*>(a.out) + (static_cast<size_t>(i) * a.Hq + x.head) * (kD * 2);

@@ -113,8 +113,8 @@ cudaError_t prepare_attn_f32();  // opt in to the kernel's dynamic shared memory
 cudaError_t launch_attn_f32(const F32Args& args, int grid, cudaStream_t stream);
 
 // Text decoder attention: causal, a local window (0: none), grouped-query heads; bf16,
-// head size 128.  Units are 128 query rows of one (segment, query head).
-constexpr int kSwaBlockRows = 128;
+// head size 128.  Units are 256 query rows (two Q tiles) of one (segment, query head).
+constexpr int kSwaBlockRows = 256;
 constexpr int kSwaHeadDim = 128;
 struct SwaArgs {
   void* out;

@@ -320,7 +320,7 @@ vt_status swa_impl(const void* q, const void* k, const void* v, void* out, const
   a.window = window;
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const long long units = vt::max_work_entries(T, n, vt::kSwaBlockRows) * static_cast<long long>(Hq);
-  const long long cap = 2ll * di->num_sms;  // two CTAs per SM
+  const long long cap = di->num_sms;  // one CTA per SM
   const int grid = static_cast<int>(units < cap ? units : cap);
   return vt::launch_attn_swa(tq, tk, tv, a, grid, stream) == cudaSuccess ? VT_OK : VT_ERR_CUDA;
 }
