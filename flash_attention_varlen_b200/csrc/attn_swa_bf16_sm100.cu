@@ -10,8 +10,8 @@
 // One CTA per SM works through units of 256 query rows of one (segment, query head): two
 // 128-row Q tiles that share every K/V tile, as in the vision kernel, so the tensor core
 // works on one tile while the other is in its softmax.  A unit visits only the key tiles its
-// rows can see (from the window start of its first row to its last row); a tile that one Q
-// tile cannot see at all costs that tile's MMAs and a masked softmax pass.
+// rows can see (from the window start of its first row to its last row), and each Q tile
+// skips a key tile none of its rows can see.
 //
 //   warp 8 (loader)  : TMA loads of the two Q tiles and of each K and V tile into 2-stage
 //                      rings (64-byte swizzle, four 32-column chunks).
@@ -68,6 +68,9 @@ struct Unit {
   int head, kv_head, q0, seg_start, seg_end;
   int j0, nkv;  // first key tile (from the segment start) and the tile count
   bool has_q1;  // the second Q tile holds rows of the segment
+  // key tiles [first[i], last[i]] of the unit that Q tile i can see: a key tile none of
+  // its rows can see (the last one for tile 0, a window-edge one for tile 1) is skipped
+  int first[2], last[2];
 };
 
 // This CTA's units: a snake over the CTAs, entry-major with the query heads inner (the
@@ -92,6 +95,13 @@ struct Units {
     const int lo = window > 0 ? max(we.seg_start, x->q0 - window + 1) : we.seg_start;
     x->j0 = (lo - we.seg_start) / kBN;
     x->nkv = (q_last - we.seg_start) / kBN - x->j0 + 1;
+    // tile 0: rows q0 .. min(q0 + 127, end - 1), from the unit's first key tile
+    x->first[0] = 0;
+    x->last[0] = (min(x->q0 + kBM, we.seg_end) - 1 - we.seg_start) / kBN - x->j0;
+    // tile 1: rows q0 + 128 .., to the unit's last key tile
+    const int lo1 = window > 0 ? max(we.seg_start, x->q0 + kBM - window + 1) : we.seg_start;
+    x->first[1] = (lo1 - we.seg_start) / kBN - x->j0;
+    x->last[1] = x->nkv - 1;
     return true;
   }
 };
@@ -263,8 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = kc % kStages;
           if (!mbar_wait_bounded(&sm.k_full[st], (kc / kStages) & 1, abort_flag, dev_status)) break;
           tc_fence_after();
-          issue_qk(T0{}, st);
-          if (x.has_q1) issue_qk(T1{}, st);
+          issue_qk(T0{}, st);  // tile 0 always sees the unit's first key tile
+          if (x.has_q1 && x.first[1] == 0) issue_qk(T1{}, st);
           mma_commit(&sm.k_empty[st]);
           ++kc;
           if (x.nkv == 1) mma_commit(&sm.q_empty);
@@ -272,21 +282,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < x.nkv; ++j, ++vc) {
           const uint32_t sv = vc % kStages;
           const bool more = j + 1 < x.nkv;
+          const bool t1 = x.has_q1 && j >= x.first[1];  // tile 1 sees key tile j
           if (!mbar_wait_bounded(&sm.v_full[sv], (vc / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
-          if (!issue_pv(T0{}, sv, j > 0)) { ok = false; break; }
-          if (!x.has_q1) mma_commit(&sm.v_empty[sv]);
+          if (j <= x.last[0] && !issue_pv(T0{}, sv, j > 0)) { ok = false; break; }
+          if (!t1) mma_commit(&sm.v_empty[sv]);
           const uint32_t st = kc % kStages;
           if (more) {
             if (!mbar_wait_bounded(&sm.k_full[st], (kc / kStages) & 1, abort_flag, dev_status)) { ok = false; break; }
             tc_fence_after();
-            issue_qk(T0{}, st);
+            if (j + 1 <= x.last[0]) issue_qk(T0{}, st);
           }
-          if (x.has_q1) {
-            if (!issue_pv(T1{}, sv, j > 0)) { ok = false; break; }
+          if (t1) {
+            if (!issue_pv(T1{}, sv, j > x.first[1])) { ok = false; break; }
             mma_commit(&sm.v_empty[sv]);
           }
           if (more) {
-            if (x.has_q1) issue_qk(T1{}, st);
+            if (x.has_q1 && j + 1 >= x.first[1]) issue_qk(T1{}, st);
             mma_commit(&sm.k_empty[st]);
             ++kc;
             if (j + 2 == x.nkv) mma_commit(&sm.q_empty);
@@ -313,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // allowed keys of row i: [lo_i, i]; none for rows past the segment end
       const int lo_i = a.window > 0 ? max(x.seg_start, i - a.window + 1) : x.seg_start;
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < x.nkv; ++j) {
+      const int ja = x.first[wg], jb = x.last[wg];
+      for (int j = ja; j <= jb; ++j) {
         if (!warp_wait(&sm.s_full[wg], s_cnt & 1, abort_flag, dev_status)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
@@ -358,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O holds this unit's earlier tiles from j = 1 on; S_j completing implies PV_{j-1}
         // has completed (one in-order MMA stream).  TMEM loads and stores are
         // warp-collective: the whole warp rescales when one of its rows needs it.
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (j > ja && __any_sync(0xffffffffu, alpha != 1.f)) {
           const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
           for (int c0 = 0; c0 < kD; c0 += 32) {
@@ -415,8 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 -> HBM
-      if (!warp_wait(&sm.o_done[wg], (o_base + x.nkv - 1) & 1, abort_flag, dev_status)) break;
-      o_base += x.nkv;
+      if (!warp_wait(&sm.o_done[wg], (o_base + (jb - ja)) & 1, abort_flag, dev_status)) break;
+      o_base += jb - ja + 1;
       tc_fence_after();
       const float inv_l = 1.0f / l;
       uint8_t* row = static_cast<uint8_t*>(a.out) + (static_cast<size_t>(i) * a.Hq + x.head) * (kD * 2);
