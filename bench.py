@@ -405,6 +405,9 @@ def oracle_per_config(outputs):
         if item[0] == "decoder":
             res[name] = decoder_vs_oracle(*item[1:])
             continue
+        if item[0] == "rope2d":
+            res[name] = rope2d_vs_oracle(*item[1:])
+            continue
         c, got = item
         q, k, v = c.inputs()
         t0 = time.perf_counter()
@@ -422,6 +425,25 @@ def oracle_per_config(outputs):
             entry["within_bound"] = bool(err.max() <= 1e-5)
         res[name] = entry
     return res
+
+
+def rope2d_vs_oracle(inputs, got):
+    """The RoPE attention output against the oracle (rotate in f64, then attention) on one
+    row of every (256-row block, head) unit, alternating ends of the block."""
+    from oracle import rope
+    q, k, v, cu, pos = inputs
+    T, H = q.shape[0], q.shape[1]
+    blocks = np.arange(0, T, 256)
+    tok = np.concatenate([blocks + (h % 2) * 255 for h in range(H)])
+    head = np.repeat(np.arange(H), len(blocks))
+    t0 = time.perf_counter()
+    ref = rope.attn_rows_rope2d(q, k, v, cu, SCALE, pos, tok, head)
+    dt = time.perf_counter() - t0
+    err = np.abs(got[tok, head] - ref)
+    return {"rows": int(len(tok)), "max_abs": float(err.max()), "mean_abs": float(err.mean()),
+            "max_abs_O": float(np.abs(ref).max()), "finite": bool(np.isfinite(got).all()),
+            "within_bound": bool(err.max() <= 1e-2 and err.mean() <= 1e-3),
+            "oracle_s_rows": round(dt, 3)}
 
 
 def decoder_vs_oracle(inputs, got):
@@ -488,6 +510,10 @@ def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3, keep_outputs=
         out["window_segmentation_128x128"] = time_window_segmentation(fa, torch, dev, calls)
     except Exception as exc:  # noqa: BLE001
         out["window_segmentation_128x128"] = {"error": str(exc)[:200]}
+    try:  # informational
+        out["rope2d_window_16x1024"] = time_rope2d(fa, torch, dev, calls, keep_outputs)
+    except Exception as exc:  # noqa: BLE001
+        out["rope2d_window_16x1024"] = {"error": str(exc)[:200]}
     for window in (workloads.DECODER_WINDOW, 0):
         name = f"decoder_{'sliding' if window else 'full'}_16384"
         try:  # informational, like the segmentation timings
@@ -495,6 +521,48 @@ def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3, keep_outputs=
         except Exception as exc:  # noqa: BLE001
             out[name] = {"error": str(exc)[:200]}
     return out
+
+
+def time_rope2d(fa, torch, dev, calls: int, keep_outputs):
+    """The tower's window layer (16 x 1024 tokens in window order) with the 2D RoPE: the
+    attention over rope(Q), rope(K) (Q rotated in the attention kernel, K by one pass) beside
+    the plain attention on the same inputs, and the K rotation pass alone in GB/s."""
+    case = workloads.tower_layer_case(0, GRID)
+    q, k, v = case.inputs()
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    dq, dk, dv = to(q), to(k), to(v)
+    do, k_rot = torch.empty_like(dq), torch.empty_like(dk)
+    cu = torch.from_numpy(case.cu_seqlens.copy()).to(dev)
+    perm, _ = fa.window_partition([(GRID, GRID)], 32, device=dev)
+    pos = torch.from_numpy(workloads.patch_positions(GRID, GRID)).to(dev)[perm.long()].contiguous()
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(calls):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        fa.check_device_status(stream)
+        return e0.elapsed_time(e1) / calls
+    plain = timed(lambda: fa.attn_fwd(dq, dk, dv, cu, scale=SCALE, out=do))
+    rope = timed(lambda: fa.attn_fwd_rope2d(dq, dk, dv, cu, pos, scale=SCALE, out=do, k_rot=k_rot))
+    kpass = timed(lambda: fa.rope2d(dk, pos, out=k_rot))
+    moved = 2 * dk.numel() * dk.element_size() + pos.numel() * pos.element_size()
+    _, hbm_peak, _ = measured_peaks()
+    gbs = moved / (kpass * 1e-3) / 1e9
+    if keep_outputs is not None:
+        keep_outputs["rope2d_window_16x1024"] = ("rope2d", (q, k, v, case.cu_seqlens, pos.cpu().numpy()),
+                                                  do.float().cpu().numpy().astype(np.float64))
+    return {"dtype": "bf16", "tokens": case.T, "segments": case.num_segments,
+            "ms_attn_rope2d": round(rope, 4), "ms_attn_plain": round(plain, 4),
+            "rope_overhead_pct": round(100.0 * (rope - plain) / plain, 1),
+            "tflops_attn_rope2d": round(case.flops() / (rope * 1e-3) / 1e12, 2),
+            "ms_k_rotation": round(kpass, 4), "k_rotation_gbs": round(gbs, 1),
+            "k_rotation_frac_of_hbm_peak": round(gbs / hbm_peak, 3) if hbm_peak else None}
 
 
 def time_decoder(fa, torch, dev, window: int, calls: int, keep_outputs, name: str):

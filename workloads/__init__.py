@@ -160,6 +160,13 @@ def flops(cu_seqlens, H: int = HEADS, D: int = HEAD_DIM) -> int:
     return int(4 * int((L * L).sum()) * H * D)
 
 
+def patch_positions(grid_h: int, grid_w: int) -> np.ndarray:
+    """int32 [grid_h * grid_w, 2]: each patch's 1-based (column + 1, row + 1) in row-major
+    patch order, the positions a 2D RoPE input carries."""
+    ys, xs = np.meshgrid(np.arange(grid_h), np.arange(grid_w), indexing="ij")
+    return np.stack([xs.ravel() + 1, ys.ravel() + 1], axis=1).astype(np.int32)
+
+
 # Text decoder attention (the Muse Glimmer next-steps document, "Architecture / Text
 # decoder"): 32 query heads over 2 key/value heads, head size 128, local window 2048.
 DECODER_HQ, DECODER_HKV, DECODER_D, DECODER_WINDOW = 32, 2, 128, 2048
