@@ -525,8 +525,9 @@ def time_configs(fa, torch, dev, calls: int = 20, warmup: int = 3, keep_outputs=
 
 def time_rope2d(fa, torch, dev, calls: int, keep_outputs):
     """The tower's window layer (16 x 1024 tokens in window order) with the 2D RoPE: the
-    attention over rope(Q), rope(K) (Q rotated in the attention kernel, K by one pass) beside
-    the plain attention on the same inputs, and the K rotation pass alone in GB/s."""
+    attention over rope(Q), rope(K) (one pass rotates both, then the attention) beside the
+    plain attention on the same inputs, and the rotation pass over K alone in GB/s, timed
+    as a CUDA graph of 20 passes so the host's per-call cost does not hide in it."""
     case = workloads.tower_layer_case(0, GRID)
     q, k, v = case.inputs()
     to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -550,7 +551,17 @@ def time_rope2d(fa, torch, dev, calls: int, keep_outputs):
         return e0.elapsed_time(e1) / calls
     plain = timed(lambda: fa.attn_fwd(dq, dk, dv, cu, scale=SCALE, out=do))
     rope = timed(lambda: fa.attn_fwd_rope2d(dq, dk, dv, cu, pos, scale=SCALE, out=do, k_rot=k_rot))
-    kpass = timed(lambda: fa.rope2d(dk, pos, out=k_rot))
+    side = torch.cuda.Stream(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        fa.rope2d(dk, pos, out=k_rot, stream=side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(20):
+                fa.rope2d(dk, pos, out=k_rot, stream=side)
+    torch.cuda.synchronize(dev)
+    kpass = timed(graph.replay) / 20
+    del graph
     moved = 2 * dk.numel() * dk.element_size() + pos.numel() * pos.element_size()
     _, hbm_peak, _ = measured_peaks()
     gbs = moved / (kpass * 1e-3) / 1e9

@@ -196,9 +196,9 @@ def attn_fwd_rope2d(q, k, v, cu_seqlens, pos, theta: float = 10000.0, scale: flo
                     out=None, k_rot=None, stream=None):
     """Block-diagonal attention over rope(Q), rope(K), V (bf16 [T, H, 96] CUDA tensors).
 
-    pos: int32 [T, 2] CUDA tensor of 1-based (pw, ph) per token.  Q is rotated inside the
-    kernel; K is rotated into ``k_rot`` (a new tensor unless given; ``k_rot=k`` rotates
-    in place).  Returns ``out``.
+    pos: int32 [T, 2] CUDA tensor of 1-based (pw, ph) per token.  One pass rotates Q into
+    ``out`` and K into ``k_rot`` (a new tensor unless given; ``k_rot=k`` rotates in place);
+    the attention then reads Q from ``out`` and writes O over it.  Returns ``out``.
     """
     import torch
     if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:

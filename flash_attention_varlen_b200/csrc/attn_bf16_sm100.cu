@@ -10,7 +10,7 @@
 // one (segment, head): two 128-row Q tiles that share every K/V tile.
 //
 //   warps 8-11         : warp 8 loads K/V, warp 9 issues MMAs, warp 10 loads Q, warp 11
-//                        rotates Q by the 2D RoPE when the call asks for it
+//                        has no role (it completes the third warpgroup)
 //   warp 8  (K/V loader): TMA loads of K/V tiles into a 2-stage ring (64-byte
 //                        swizzled, 32-column chunks).
 //   warp 10 (Q loader) : TMA loads of Q0/Q1 into a double buffer, so the next
@@ -22,8 +22,6 @@
 //                        tensor core works on one tile while the other is in softmax;
 //                        one flat stream over all units of the CTA, so a tile's first
 //                        S of the next unit follows its own last PV of this one.
-//   warp 11 (RoPE)     : only with a RoPE call: rotates each landed Q tile in shared
-//                        memory (2D RoPE, width first) before its QKs may read it.
 //   warps 0-3, 4-7     : softmax warpgroups for Q0 and Q1, one thread per row:
 //                        tcgen05.ld of the S row, row max (three-input max tree),
 //                        p = 2^(s*c - m) (packed f32x2 FMA, then MUFU ex2 for two
@@ -50,7 +48,6 @@
 // bounded and an abort flag lets all roles leave together.
 #include "internal.h"
 #include "ptx.cuh"
-#include "rope2d.cuh"
 
 namespace vt {
 namespace {
@@ -74,7 +71,7 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "regi
 constexpr int kWarpLoad = 8;       // K/V loader
 constexpr int kWarpMma = 9;
 constexpr int kWarpLoadQ = 10;     // Q loader (runs up to one unit ahead)
-constexpr int kWarpRope = 11;      // 2D RoPE of the Q tiles (when enabled)
+// Warp 11 has no role: the block keeps three full warpgroups for the register split.
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 // The running max only moves when a tile's max exceeds it by more than this (log2
@@ -115,7 +112,6 @@ struct Smem {
   uint8_t v[kVStages][kVTileBytes];
   uint64_t q_full[kQBufs][2];
   uint64_t q_empty[kQBufs];
-  uint64_t q_ready[kQBufs][2];  // RoPE prologue: the landed Q tile has been rotated
   uint64_t k_full[kKStages];
   uint64_t k_empty[kKStages];
   uint64_t v_full[kVStages];
@@ -279,34 +275,6 @@ __device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint
     tma_load_3d(static_cast<uint8_t*>(dst) + c * kChunkBytes, map, bar, c * 32, head, row0);
 }
 
-// 2D RoPE of one landed 128-row Q tile in shared memory (three 32-column chunks, 64-byte
-// swizzle: 16-byte unit u of row r sits at unit u ^ ((r >> 1) & 3)), by one warp: lane l
-// rotates rows l, l + 32, l + 64, l + 96, each as six (group, group + 6) pairs of 16-byte
-// groups (columns 8g .. 8g + 7 with 48 + 8g .. 48 + 8g + 7).  Rows past the segment end
-// are left as they are: they are computed but never stored.
-__device__ __forceinline__ void rope_q_tile(uint8_t* tile, const int32_t* pos, int row_tok0,
-                                            int seg_end, const float* freq, int lane) {
-#pragma unroll 1
-  for (int k = 0; k < 4; ++k) {
-    const int r = lane + 32 * k;
-    const int tok = row_tok0 + r;
-    if (tok >= seg_end) continue;
-    const int2 p = __ldg(reinterpret_cast<const int2*>(pos) + tok);
-    const float pw = static_cast<float>(p.x), ph = static_cast<float>(p.y);
-    const uint32_t sw = (r >> 1) & 3;
-#pragma unroll 1
-    for (int g = 0; g < 6; ++g) {
-      const int g2 = g + 6;
-      uint4* plo = reinterpret_cast<uint4*>(tile + (g >> 2) * kChunkBytes + r * 64 + (((g & 3) ^ sw) << 4));
-      uint4* phi = reinterpret_cast<uint4*>(tile + (g2 >> 2) * kChunkBytes + r * 64 + (((g2 & 3) ^ sw) << 4));
-      uint4 lo = *plo, hi = *phi;
-      rope_rotate_group(lo, hi, g, pw, ph, freq);
-      *plo = lo;
-      *phi = hi;
-    }
-  }
-}
-
 // Builds the shared-memory work table of a call with n <= kInlineSegments segments, by one
 // warp: the same validation (cu[0] == 0, cu[n] == T, no negative length), the same
 // longest-first order (ties by index) and the same unit order flag as the scheduling
@@ -389,8 +357,7 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
   uint32_t kv_it = 0, unit_it = 0, p_cnt0 = 0, p_cnt1 = 0;
   uint32_t q1_it0 = 0, q1_it1 = 0;  // Q1 loads consumed per buffer
   // Q of unit number n (buffer n % kQBufs) has landed
-  // (with the RoPE prologue: has been rotated in shared memory)
-  uint64_t(*qbar)[2] = a.rope_pos != nullptr ? sm.q_ready : sm.q_full;
+  uint64_t(*qbar)[2] = sm.q_full;
   auto wait_q = [&](const Unit& u, uint32_t n) {
     const uint32_t b = n % kQBufs;
     if (!mma_wait(&qbar[b][0], (n / kQBufs) & 1, abort_flag, dev_status)) return false;
@@ -496,7 +463,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       for (int b = 0; b < kQBufs; ++b) {
         mbar_init(&sm.q_full[b][i], 1);
-        mbar_init(&sm.q_ready[b][i], 1);
       }
       mbar_init(&sm.s_full[i], 1);
       for (int c = 0; c < kPChunks; ++c) mbar_init(&sm.p_full[i][c], kBM);
@@ -641,27 +607,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       mma_role(sm, a, tmem, tab, E, total, order, abort_flag, dev_status);
-    }
-   } else if (warp == kWarpRope && a.rope_pos != nullptr) {
-    // ------------------------------------------------------------ RoPE prologue of Q
-    // Each Q tile is rotated once, right after it lands; the loader runs a unit ahead, so
-    // this stays ahead of the QKs that read the tile (they wait on q_ready).  The Q buffer
-    // is only refilled after those QKs completed (q_empty), i.e. after this rotation.
-    uint32_t unit_it = 0, q1a = 0, q1b = 0;
-    for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid(); ++unit_it) {
-      const Unit x = us.take();
-      const uint32_t b = unit_it % kQBufs;
-      bool ok = true;
-      for (int i = 0; i < (x.has_q1 ? 2 : 1); ++i) {
-        const uint32_t parity = i == 0 ? (unit_it / kQBufs) & 1 : (b ? q1b : q1a) & 1;
-        if (!warp_wait(&sm.q_full[b][i], parity, abort_flag, dev_status)) { ok = false; break; }
-        rope_q_tile(sm.q[b][i], a.rope_pos, x.q0 + i * kBM, x.seg_end, a.rope.f, lane);
-        fence_proxy_async_smem();  // the rotated tile is read by the tensor core (async proxy)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.q_ready[b][i]);
-      }
-      if (!ok) break;
-      if (x.has_q1) { if (b) ++q1b; else ++q1a; }
     }
    }
   } else {

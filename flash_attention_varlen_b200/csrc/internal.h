@@ -62,9 +62,13 @@ struct RopeFreqs {
   float f[24];
 };
 RopeFreqs rope_freqs(double theta);
-// out = rope(x) for bf16 [T, H, 96] (out may equal x); pos: int32 [T][2] 1-based (pw, ph).
-cudaError_t launch_rope2d(const void* x, void* out, const int32_t* pos, int32_t T, int32_t H,
-                          const RopeFreqs& f, int num_sms, cudaStream_t stream);
+// out[i] = rope(x[i]) for count (1 or 2) bf16 [T, H, 96] tensors in one launch (out[i] may
+// equal x[i]); pos: int32 [T][2] 1-based (pw, ph), shared by the tensors.  The kernel lets
+// a dependent launch (programmatic stream serialization) start early.
+constexpr int kRopeMaxTensors = 2;
+cudaError_t launch_rope2d(const void* const* x, void* const* out, int count, const int32_t* pos,
+                          int32_t T, int32_t H, const RopeFreqs& f, int num_sms,
+                          cudaStream_t stream);
 
 // bf16 forward on tcgen05 tensor cores (sm_100a).
 constexpr int kBf16BlockRows = 256;  // two 128-row Q tiles per unit
@@ -84,10 +88,6 @@ struct Bf16Args {
   // > 0 only in the failure-path self-test: the MMA thread first waits this many cycles
   // on a barrier that never completes (see vt_attn_selftest_wait_timeout)
   int32_t stall_test_cycles = 0;
-  // 2D RoPE prologue: when rope_pos (device int32 [T][2], 1-based (pw, ph)) is set, every
-  // Q tile is rotated in shared memory after it lands and before any QK reads it
-  const int32_t* rope_pos = nullptr;
-  RopeFreqs rope;
 };
 size_t bf16_smem_bytes();
 cudaError_t prepare_attn_bf16();  // opt in to the kernel's dynamic shared memory (per device)
@@ -142,8 +142,6 @@ struct FwdCall {
   int dtype;  // vt_dtype
   cudaStream_t stream;
   int32_t stall_test_cycles;  // > 0 only for the bf16 failure-path self-test
-  const int32_t* rope_pos = nullptr;  // bf16 only: rotate Q by the 2D RoPE in the kernel
-  float rope_theta = 10000.0f;
 };
 
 // Host-side argument checks shared by every forward entry point; touches no device.

@@ -31,11 +31,13 @@ __device__ __forceinline__ void rope_sincos(float x, float* s, float* c) {
   __sincosf(r, s, c);
 }
 
-// Rotate the 8 pairs of one 16-byte group: lo holds columns 8u .. 8u+7 (u < 6, the first
-// half), hi the columns 48 + 8u .. 48 + 8u + 7; pw, ph are the token's 1-based positions
-// and freq the D/4 frequencies.  Values are bf16, rounded to nearest-even after rotation.
-__device__ __forceinline__ void rope_rotate_group(uint4& lo, uint4& hi, int u, float pw, float ph,
-                                                  const float* freq) {
+// Rotate the 8 pairs of one 16-byte group by one axis position p: lo holds columns
+// 8u .. 8u+7 of the first half (u < 6), hi the columns 48 + 8u .. 48 + 8u + 7, and f8 the
+// group's 8 frequencies.  D/4 = 24 is a multiple of 8, so all 8 columns of a group lie on
+// one axis: groups 0-2 take the width position with f_{8u+j}, groups 3-5 the height
+// position with f_{8(u-3)+j}.  Values are bf16, rounded to nearest-even after rotation.
+template <typename Freqs>
+__device__ __forceinline__ void rope_rotate8(uint4& lo, uint4& hi, float p, const Freqs& f8) {
   uint32_t a[4] = {lo.x, lo.y, lo.z, lo.w};
   uint32_t b[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
@@ -48,10 +50,8 @@ __device__ __forceinline__ void rope_rotate_group(uint4& lo, uint4& hi, int u, f
     float y0[2], y1[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const int d = 8 * u + 2 * e + k;  // column in the first half, 0 .. 47
-      const float ang = d < kRopeFreqs ? pw * freq[d] : ph * freq[d - kRopeFreqs];
       float sn, cs;
-      rope_sincos(ang, &sn, &cs);
+      rope_sincos(p * f8[2 * e + k], &sn, &cs);
       y0[k] = fmaf(x0[k], cs, -x1[k] * sn);
       y1[k] = fmaf(x1[k], cs, x0[k] * sn);
     }
@@ -63,6 +63,12 @@ __device__ __forceinline__ void rope_rotate_group(uint4& lo, uint4& hi, int u, f
   }
   lo = make_uint4(a[0], a[1], a[2], a[3]);
   hi = make_uint4(b[0], b[1], b[2], b[3]);
+}
+
+// The same for group u of a token at 1-based positions (pw, ph), freq the D/4 frequencies.
+__device__ __forceinline__ void rope_rotate_group(uint4& lo, uint4& hi, int u, float pw, float ph,
+                                                  const float* freq) {
+  rope_rotate8(lo, hi, u < 3 ? pw : ph, freq + 8 * (u < 3 ? u : u - 3));
 }
 
 }  // namespace vt

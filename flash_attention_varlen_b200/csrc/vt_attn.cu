@@ -232,10 +232,6 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) 
     a.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(c.scale)) * log2e);
     a.idesc_qk = make_idesc_bf16(128, 128, false, false, c.scale < 0.0f);
     a.stall_test_cycles = c.stall_test_cycles;
-    if (c.rope_pos != nullptr) {
-      a.rope_pos = c.rope_pos;
-      a.rope = rope_freqs(c.rope_theta);
-    }
     const int grid = static_cast<int>(max_units < di->num_sms ? max_units : di->num_sms);
     if (launch_attn_bf16(tq, tk, tv, a, grid, c.stream) != cudaSuccess) return VT_ERR_CUDA;
   } else {
@@ -469,17 +465,25 @@ vt_status vt_attn_fwd_rope2d(const void* q, const void* k, const void* v, void* 
   if ((reinterpret_cast<uintptr_t>(k) & 15u) || (reinterpret_cast<uintptr_t>(pos) & 7u))
     return VT_ERR_INVALID_ARG;
   const size_t bytes = static_cast<size_t>(total_tokens) * H * D * 2;
+  const size_t pos_bytes = static_cast<size_t>(total_tokens) * 2 * sizeof(int32_t);
   if (k != k_rot && (ranges_overlap(k, bytes, k_rot, bytes) || ranges_overlap(k, bytes, out, bytes)))
     return VT_ERR_INVALID_ARG;
   if (ranges_overlap(k_rot, bytes, q, bytes) || ranges_overlap(k_rot, bytes, v, bytes))
     return VT_ERR_INVALID_ARG;
-  // K is rotated once by the HBM-bound pass (each K tile is read by every unit of its
-  // segment, so rotating it there would repeat the work per unit); Q is rotated inside the
-  // attention kernel, once per unit, after its tile lands in shared memory.
-  st = vt_rope2d(k, k_rot, pos, total_tokens, H, D, theta, stream_ptr);
-  if (st != VT_OK) return st;
-  c.rope_pos = pos;
-  c.rope_theta = theta;
+  if (ranges_overlap(pos, pos_bytes, out, bytes) || ranges_overlap(pos, pos_bytes, k_rot, bytes))
+    return VT_ERR_INVALID_ARG;
+  const int nsm = sm_count();
+  if (nsm < 1) return VT_ERR_CUDA;
+  // One HBM-bound pass rotates Q into `out` and K into k_rot; the attention then reads its
+  // Q from `out` and writes O over it.  Each unit of the kernel reads its own Q rows once,
+  // before any of its O rows are stored, and no other unit reads those rows: rows a Q tile
+  // carries past its segment's end belong to another unit, and their results are dropped.
+  const void* src[2] = {q, k};
+  void* dst[2] = {out, k_rot};
+  if (vt::launch_rope2d(src, dst, 2, pos, total_tokens, H, vt::rope_freqs(theta), nsm,
+                        static_cast<cudaStream_t>(stream_ptr)) != cudaSuccess)
+    return VT_ERR_CUDA;
+  c.q = out;
   return fwd_impl(c);
 }
 
@@ -521,9 +525,11 @@ vt_status vt_rope2d(const void* x, void* out, const int32_t* pos, int32_t total_
     return VT_ERR_INVALID_ARG;
   const size_t bytes = static_cast<size_t>(total_tokens) * H * D * 2;
   if (x != out && ranges_overlap(x, bytes, out, bytes)) return VT_ERR_INVALID_ARG;
+  if (ranges_overlap(pos, static_cast<size_t>(total_tokens) * 2 * sizeof(int32_t), out, bytes))
+    return VT_ERR_INVALID_ARG;
   const int nsm = sm_count();
   if (nsm < 1) return VT_ERR_CUDA;
-  return vt::launch_rope2d(x, out, pos, total_tokens, H, vt::rope_freqs(theta), nsm,
+  return vt::launch_rope2d(&x, &out, 1, pos, total_tokens, H, vt::rope_freqs(theta), nsm,
                            static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? VT_OK
              : VT_ERR_CUDA;

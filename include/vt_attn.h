@@ -239,7 +239,7 @@ vt_status vt_permute_rows_check(void* stream);
  *   element d < D/2 pairs with d + D/2: (x_d, x_{d+D/2}) turns by a_d.
  * Arithmetic in f32 (sin/cos after reduction to [-pi, pi]); the result is rounded to bf16.
  *   x, out   device pointers, 16-byte aligned; out == x rotates in place, otherwise the
- *            two must not overlap.
+ *            two must not overlap; pos must not overlap out.
  *   D        only 96 (VT_ERR_UNSUPPORTED otherwise); H >= 1; theta finite and > 0 (the
  *            tower's base: 10000).
  * Asynchronous on `stream`; total_tokens == 0 is a no-op.
@@ -257,11 +257,15 @@ vt_status vt_rope2d(const void* x, void* out, const int32_t* pos, int32_t total_
  *   k_rot   caller-owned device buffer [total_tokens, H, D] bf16, 16-byte aligned, that
  *           receives rope(K) (the attention reads K from it); k_rot == k rotates K in
  *           place.  It must not overlap q, v or out.
- * Q is rotated inside the attention kernel: each 128-row Q tile once, in shared memory,
- * right after it lands and before the QK products read it (the fused RoPE prologue).  K
- * is rotated by one HBM-bound vt_rope2d pass queued first on the same stream: every K tile
- * is read by all units of its segment, so rotating it inside the kernel would repeat the
- * rotation once per unit.  Errors and asynchrony as for vt_attn_fwd.
+ *   out     as for vt_attn_fwd; it also holds rope(Q) between the two steps below, so on
+ *           an error reported by the device its contents are undefined.  pos must not
+ *           overlap out or k_rot.
+ * Two launches on `stream`: one HBM-bound pass (vt_rope2d's arithmetic) rotates Q into out
+ * and K into k_rot; the attention kernel then reads Q from out and writes O over it (each
+ * unit of the kernel reads its own Q rows before it stores those rows of O, and no other
+ * unit needs them).  With at most 32 segments the attention kernel follows the pass
+ * directly and, launched with programmatic stream serialization, sets itself up while the
+ * pass ends.  Errors and asynchrony as for vt_attn_fwd.
  */
 vt_status vt_attn_fwd_rope2d(const void* q, const void* k, const void* v, void* out,
                              const int32_t* cu_seqlens, int32_t num_segments, int32_t total_tokens,

@@ -178,3 +178,49 @@ def test_rope_attention_positions_all_equal_is_plain_attention():
     pos = np.repeat(np.array([[7, 3], [60, 1], [1, 128]], np.int32), lengths, axis=0)
     got, _ = _rope_attn(q, k, v, cu, pos)
     _check(got, oracle.attn_fwd(q, k, v, cu, 1.0 / math.sqrt(96)), "rope equal positions")
+
+
+@pytest.mark.parametrize("case", ["window16x1024", "ragged"])
+def test_rope_attention_equals_rotation_then_plain_attention_bit_for_bit(case):
+    """The RoPE attention rotates Q into ``out`` and the attention writes O over it: the
+    result must equal, bit for bit, rope2d(Q), rope2d(K) into separate buffers followed by
+    the plain attention.  The ragged case ends segments inside Q tiles, where a tile also
+    carries rows of the next segment that another unit overwrites with its O."""
+    import math
+    import flash_attention_varlen_b200 as fa
+    if case == "window16x1024":
+        perm, cu = window_permutation([(128, 128)], 32)
+        pos = rope.image_positions([(128, 128)])[perm]
+    else:
+        lengths = [1, 200, 129, 383, 2, 640, 255, 90]
+        cu = workloads.cu_from_lengths(lengths)
+        rng = np.random.default_rng(8)
+        pos = rng.integers(1, 129, size=(int(cu[-1]), 2)).astype(np.int32)
+    T = int(cu[-1])
+    q, k, v = workloads.qkv(37, T)
+    dq, dk, dv = _bf16_dev(q), _bf16_dev(k), _bf16_dev(v)
+    dcu = torch.from_numpy(np.ascontiguousarray(cu, np.int32)).cuda()
+    dpos = torch.from_numpy(np.ascontiguousarray(pos, np.int32)).cuda()
+    scale = 1.0 / math.sqrt(96)
+    fused = fa.attn_fwd_rope2d(dq, dk, dv, dcu, dpos, scale=scale)
+    qr, kr = fa.rope2d(dq, dpos), fa.rope2d(dk, dpos)
+    steps = fa.attn_fwd(qr, kr, dv, dcu, scale=scale)
+    fa.check_device_status()
+    assert torch.equal(fused, steps)
+    assert torch.equal(dq, _bf16_dev(q))  # Q itself is left as it was
+
+
+def test_rope_attention_many_images_with_the_scheduling_prepass():
+    """40 small images (more segments than the kernel schedules by itself, so the
+    scheduling prepass runs between the rotation pass and the attention), every element
+    against the RoPE oracle."""
+    import math
+    rng = np.random.default_rng(9)
+    grids = [(int(h), int(w)) for h, w in rng.integers(2, 19, size=(40, 2))]
+    pos = rope.image_positions(grids)
+    cu = workloads.cu_from_lengths([h * w for h, w in grids])
+    T = int(cu[-1])
+    q, k, v = workloads.qkv(38, T)
+    got, _ = _rope_attn(q, k, v, cu, pos)
+    ref = rope.attn_fwd_rope2d(q, k, v, cu, 1.0 / math.sqrt(96), pos)
+    _check(got, ref, "rope 40 images")
