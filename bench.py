@@ -92,8 +92,10 @@ def measured_peaks():
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return float(d["bf16_tflops"]), float(d.get("hbm_gbs", 0.0)), "measured (burst)"
-    return 1590.0, 6650.0, "fallback"
+        return (float(d["bf16_tflops"]), float(d.get("hbm_gbs", 0.0)),
+                "measured burst dense bf16 (MEASURED_PEAKS.json bf16_tflops)")
+    return 1590.0, 6650.0, ("fallback: 1.59 PFLOP/s dense bf16 and 6.65 TB/s, an earlier "
+                            "measurement on this pool (MEASURED_PEAKS.json absent)")
 
 
 def kernel_sha() -> str:
@@ -357,7 +359,7 @@ def run_ours(args):
             "peak": peak,
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "peak_source": f"{peak_src} dense bf16 (MEASURED_PEAKS.json bf16_tflops)",
+            "peak_source": peak_src,
             "traffic": traffic,
             "kernel": "attn_bf16_kernel (calls of at most 32 segments, as in the tower, schedule themselves; a prepass would be timed with its call)",
             "per_launch": "4*sum(L^2)*H*D FLOPs of the call / CUDA-event duration of the call, "

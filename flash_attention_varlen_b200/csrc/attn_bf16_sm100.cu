@@ -10,7 +10,7 @@
 // one (segment, head): two 128-row Q tiles that share every K/V tile.
 //
 //   warps 8-11         : warp 8 loads K/V, warp 9 issues MMAs, warp 10 loads Q, warp 11
-//                        has no role (it completes the third warpgroup)
+//                        stores finished O tiles (staged-epilogue instantiation only)
 //   warp 8  (K/V loader): TMA loads of K/V tiles into a 2-stage ring (64-byte
 //                        swizzled, 32-column chunks).
 //   warp 10 (Q loader) : TMA loads of Q0/Q1 into a double buffer, so the next
@@ -30,7 +30,11 @@
 //                        moves when the new tile max exceeds it by more than a
 //                        threshold, so O in TMEM is rarely touched), P packed to
 //                        bf16 and written back over S in TMEM, then the epilogue
-//                        O / l -> bf16 -> HBM.
+//                        O / l -> bf16, stored row by row by each thread; or, in the
+//                        staged instantiation (calls of many short units), a whole
+//                        128-row tile is staged in the unit's Q buffer (its QKs are
+//                        done) and warp 11 sends it out with TMA stores, while the
+//                        rows of a tile cut by its segment's end still go row by row.
 //
 // CTAs take their units in a longest-first snake order (see UnitStream).
 //
@@ -71,7 +75,7 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "regi
 constexpr int kWarpLoad = 8;       // K/V loader
 constexpr int kWarpMma = 9;
 constexpr int kWarpLoadQ = 10;     // Q loader (runs up to one unit ahead)
-// Warp 11 has no role: the block keeps three full warpgroups for the register split.
+constexpr int kWarpStore = 11;     // TMA stores of the O tiles staged in the Q buffers
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
 // The running max only moves when a tile's max exceeds it by more than this (log2
@@ -112,6 +116,11 @@ struct Smem {
   uint8_t v[kVStages][kVTileBytes];
   uint64_t q_full[kQBufs][2];
   uint64_t q_empty[kQBufs];
+  uint64_t q_free[kQBufs];  // the O tiles staged in this Q buffer have been read out
+  // tile i's 128 O rows are staged in Q buffer b.  One barrier per buffer: staging into b
+  // again needs the Q of the unit two on, which is loaded only after b's stores were read,
+  // so a barrier never runs a phase ahead of the store warp's wait.
+  uint64_t o_staged[kQBufs][2];
   uint64_t k_full[kKStages];
   uint64_t k_empty[kKStages];
   uint64_t v_full[kVStages];
@@ -448,9 +457,14 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
   mbar_wait_drain(&sm.drain, 0);
 }
 
+// kStageO: whole O tiles leave through the Q buffers and TMA stores (warp 11), else every
+// row is stored by its thread and warp 11 idles.  Two instantiations, because the staging
+// code alone, never run, moved the softmax loop's code enough to cost ~1.5% on long units.
+template <bool kStageO>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ Bf16Args a) {
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                     const __grid_constant__ Bf16Args a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (raw & 1023u)) & 1023u));
@@ -468,7 +482,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < kPChunks; ++c) mbar_init(&sm.p_full[i][c], kBM);
       mbar_init(&sm.o_done[i], 1);
     }
-    for (int b = 0; b < kQBufs; ++b) mbar_init(&sm.q_empty[b], 1);
+    for (int b = 0; b < kQBufs; ++b) {
+      mbar_init(&sm.q_empty[b], 1);
+      mbar_init(&sm.q_free[b], 1);
+    }
+    for (int b = 0; b < kQBufs; ++b)
+      for (int i = 0; i < 2; ++i) mbar_init(&sm.o_staged[b][i], kBM);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -583,8 +602,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid(); ++unit_it) {
         const Unit x = us.take();
         const uint32_t b = unit_it % kQBufs, use = unit_it / kQBufs;
-        // buffer b is free once every QK of the unit that used it before has completed
-        if (use > 0 && !mbar_wait_bounded(&sm.q_empty[b], (use - 1) & 1, abort_flag, dev_status))
+        // buffer b is free once every QK of the unit that used it before has completed and
+        // the O tiles that unit staged in it have been stored
+        if (use > 0 && (!mbar_wait_bounded(&sm.q_empty[b], (use - 1) & 1, abort_flag, dev_status) ||
+                        (kStageO &&
+                         !mbar_wait_bounded(&sm.q_free[b], (use - 1) & 1, abort_flag, dev_status))))
           break;
         mbar_arrive_expect_tx(&sm.q_full[b][0], kTileBytes);
         tma_tile(sm.q[b][0], &tq, &sm.q_full[b][0], x.head, x.q0);
@@ -608,6 +630,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       mma_role(sm, a, tmem, tab, E, total, order, abort_flag, dev_status);
     }
+   } else if (kStageO && warp == kWarpStore) {
+    // ------------------------------------------------------------ O tile stores
+    // A whole 128-row O tile is staged by its softmax warpgroup in the unit's Q buffer
+    // (free once the unit's last QK has run; same layout as the Q tile) and leaves by three
+    // TMA stores.  Buffer b is released to the Q loader (q_free) once those stores have
+    // read it; a unit with nothing staged releases it at once.  This thread first waits
+    // for the unit's Q to land: the loader has then passed its q_free wait for the unit
+    // that used b before, so each arrival completes the phase the loader waits on next.
+    if (lane == 0) {
+      uint32_t unit_it = 0, staged = 0;  // bit 2b + i: parity of (buffer b, tile i) stagings
+      bool ok = true;
+      for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid() && ok; ++unit_it) {
+        const Unit x = us.take();
+        const uint32_t b = unit_it % kQBufs;
+        if (!mbar_wait_bounded(&sm.q_full[b][0], (unit_it / kQBufs) & 1, abort_flag, dev_status)) break;
+        bool issued = false;
+        for (int i = 0; i < (x.has_q1 ? 2 : 1); ++i) {
+          const int row0 = x.q0 + i * kBM;
+          if (row0 + kBM > x.seg_end) continue;  // a partial tile is stored row by row
+          const uint32_t bit = 1u << (2 * b + i);
+          if (!mbar_wait_bounded(&sm.o_staged[b][i], (staged & bit) ? 1u : 0u, abort_flag, dev_status)) {
+            ok = false;
+            break;
+          }
+          staged ^= bit;
+#pragma unroll
+          for (int c = 0; c < kD / 32; ++c)
+            tma_store_3d(&to, sm.q[b][i] + c * kChunkBytes, c * 32, x.head, row0);
+          issued = true;
+        }
+        if (!ok) break;
+        if (issued) {
+          bulk_commit_group();
+          bulk_wait_read_all();
+        }
+        mbar_arrive(&sm.q_free[b]);
+      }
+      // Shared memory stays valid until every store has read it (stores issued before an
+      // abort are still uncommitted); the grid's completion covers their global writes.
+      bulk_commit_group();
+      bulk_wait_read_all();
+    }
    }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
@@ -618,9 +682,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_base + (wg ? kColS1 : kColS0);
     const uint32_t tO = tmem + lane_base + (wg ? kColO1 : kColO0);
     const float c = a.scale_log2;
-    uint32_t s_cnt = 0, o_base = 0;
+    uint32_t s_cnt = 0, o_base = 0, unit_it = 0;
     for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid();) {
       const Unit x = us.take();
+      const uint32_t b = unit_it++ % kQBufs;
       if (wg == 1 && !x.has_q1) continue;
       const int row_tok = x.q0 + wg * kBM + r;
       float m = 0.f;
@@ -745,10 +810,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld1(tO + 96, o[96]);
       tmem_ld_wait();
       reg_fence<kD + 1>(o);
-      if (row_tok < x.seg_end) {
+      const bool whole = kStageO && x.q0 + wg * kBM + kBM <= x.seg_end;  // staged for a TMA store
+      if (whole || row_tok < x.seg_end) {
         const float inv_l = 1.0f / __uint_as_float(o[96]);
-        uint8_t* row = static_cast<uint8_t*>(a.out) +
-                       (static_cast<size_t>(row_tok) * a.H + x.head) * (kD * 2);
         const float2 il2 = make_float2(inv_l, inv_l);
         uint32_t w[kD / 2];
 #pragma unroll
@@ -756,15 +820,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 y = fmul2(make_float2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), il2);
           w[i] = pack_bf16x2(y.x, y.y);
         }
-        // a row is 192 contiguous bytes: six 32-byte stores (whole sectors) when the
-        // output is 32-byte aligned, else twelve 16-byte stores
-        if (a.out_align32) {
+        if (whole) {
+          // the row into the tile's Q buffer, in the Q tile's layout (three 32-column chunks,
+          // 16-byte unit u of row r at unit u ^ ((r >> 1) & 3)); the store warp sends it out
+          uint8_t* tile = sm.q[b][wg] + r * 64;
+          const uint32_t sw = (r >> 1) & 3;
 #pragma unroll
-          for (int i = 0; i < kD / 16; ++i) st_global_v8(row + 32 * i, w + 8 * i);
+          for (int c = 0; c < kD / 32; ++c) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint32_t* g = w + 16 * c + 4 * u;
+              *reinterpret_cast<uint4*>(tile + c * kChunkBytes + ((u ^ sw) << 4)) =
+                  make_uint4(g[0], g[1], g[2], g[3]);
+            }
+          }
+          fence_proxy_async_smem();  // generic-proxy writes, read by the TMA store
+          mbar_arrive(&sm.o_staged[b][wg]);
         } else {
+          uint8_t* row = static_cast<uint8_t*>(a.out) +
+                         (static_cast<size_t>(row_tok) * a.H + x.head) * (kD * 2);
+          // a row is 192 contiguous bytes: six 32-byte stores (whole sectors) when the
+          // output is 32-byte aligned, else twelve 16-byte stores
+          if (a.out_align32) {
 #pragma unroll
-          for (int i = 0; i < kD / 8; ++i)
-            reinterpret_cast<uint4*>(row)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            for (int i = 0; i < kD / 16; ++i) st_global_v8(row + 32 * i, w + 8 * i);
+          } else {
+#pragma unroll
+            for (int i = 0; i < kD / 8; ++i)
+              reinterpret_cast<uint4*>(row)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
         }
       }
       o_base += x.nkv;
@@ -784,7 +868,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 size_t bf16_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const Bf16Args& args, int grid, cudaStream_t stream) {
+                             const CUtensorMap& to, const Bf16Args& args, int grid,
+                             bool stage_o, cudaStream_t stream) {
   // Programmatic stream serialization: the kernel may launch while the scheduling prepass
   // before it still runs, and waits for it (griddepcontrol.wait) before reading its output.
   cudaLaunchConfig_t cfg = {};
@@ -797,11 +882,15 @@ cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_bf16_kernel, tq, tk, tv, args);
+  return stage_o ? cudaLaunchKernelEx(&cfg, attn_bf16_kernel<true>, tq, tk, tv, to, args)
+                 : cudaLaunchKernelEx(&cfg, attn_bf16_kernel<false>, tq, tk, tv, to, args);
 }
 
 cudaError_t prepare_attn_bf16() {
-  return cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const cudaError_t e = cudaFuncSetAttribute(
+      attn_bf16_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(kSmemBytes));
 }
 

@@ -91,8 +91,17 @@ struct Bf16Args {
 };
 size_t bf16_smem_bytes();
 cudaError_t prepare_attn_bf16();  // opt in to the kernel's dynamic shared memory (per device)
+// `to` maps the output like tq maps Q (same shape, box and swizzle).  With stage_o, whole
+// 128-row O tiles are staged in the unit's Q buffer and leave by TMA stores through it
+// (worth it when a CTA runs several short units: the stores overlap the next unit);
+// otherwise every row is stored by its thread.
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const Bf16Args& args, int grid, cudaStream_t stream);
+                             const CUtensorMap& to, const Bf16Args& args, int grid, bool stage_o,
+                             cudaStream_t stream);
+// The staged epilogue is chosen for calls whose segments average at most this many tokens
+// and that give each SM at least kStageMinUnitsPerSm units of 256 rows on average.
+constexpr int kStageMaxMeanSegment = 2048;
+constexpr int kStageMinUnitsPerSm = 3;
 
 // f32 forward on tcgen05 tensor cores: each operand split into three bf16 parts
 // (exactness arm).

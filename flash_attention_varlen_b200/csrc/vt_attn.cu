@@ -211,11 +211,12 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) 
   const long long max_units =
       static_cast<long long>(max_work_entries(c.total_tokens, c.num_segments, block_rows)) * c.H;
   if (c.dtype == VT_DTYPE_BF16) {
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     vt_status st;
     if ((st = make_tensor_map(&tq, c.q, c.total_tokens, c.H)) != VT_OK) return st;
     if ((st = make_tensor_map(&tk, c.k, c.total_tokens, c.H)) != VT_OK) return st;
     if ((st = make_tensor_map(&tv, c.v, c.total_tokens, c.H)) != VT_OK) return st;
+    if ((st = make_tensor_map(&to, c.out, c.total_tokens, c.H)) != VT_OK) return st;
     Bf16Args a;
     a.out = c.out;
     a.cu_seqlens = c.cu_seqlens;
@@ -233,7 +234,14 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) 
     a.idesc_qk = make_idesc_bf16(128, 128, false, false, c.scale < 0.0f);
     a.stall_test_cycles = c.stall_test_cycles;
     const int grid = static_cast<int>(max_units < di->num_sms ? max_units : di->num_sms);
-    if (launch_attn_bf16(tq, tk, tv, a, grid, c.stream) != cudaSuccess) return VT_ERR_CUDA;
+    // Staged O stores pay off when a CTA runs several short units (window layers); with
+    // one or two units per CTA the store's tail latency costs more than it hides.  The
+    // host sees only T and n (cu_seqlens stays on the device), so the rule uses the mean.
+    const int64_t rows_x_heads = static_cast<int64_t>(c.total_tokens) * c.H;
+    const bool stage_o =
+        static_cast<int64_t>(c.total_tokens) <= static_cast<int64_t>(kStageMaxMeanSegment) * c.num_segments &&
+        rows_x_heads >= static_cast<int64_t>(kStageMinUnitsPerSm) * di->num_sms * kBf16BlockRows;
+    if (launch_attn_bf16(tq, tk, tv, to, a, grid, stage_o, c.stream) != cudaSuccess) return VT_ERR_CUDA;
   } else {
     F32Args a;
     a.q = static_cast<const float*>(c.q);

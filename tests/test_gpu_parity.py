@@ -164,6 +164,18 @@ def test_ragged_segments(dtype):
     _full_case(case)
 
 
+def test_staged_output_tiles_with_ragged_segment_ends():
+    """30 segments averaging ~750 tokens with 16 heads: many 256-row units per SM, so the
+    bf16 kernel stages every whole 128-row O tile in its Q buffer and stores it by TMA,
+    while the rows of tiles cut by a segment's end (lengths off the 128 grid, a 1-token and
+    an empty segment among them) are stored row by row; every element against the oracle."""
+    lengths = [int(x) for x in workloads.uniform_int(11, 9, 26, 0, 1500)] + [1, 0, 1024, 640]
+    cu = workloads.cu_from_lengths(lengths)
+    assert int(cu[-1]) * 16 >= 3 * 148 * 256 and int(cu[-1]) <= 2048 * len(lengths)
+    case = workloads.Case("staged_ragged_bf16", cu, seed=12, dtype="bf16")
+    _full_case(case)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_more_segments_than_the_prepass_sorts(dtype):
     # 5000 segments (the prepass sorts at most 4096: more keep their given order and
