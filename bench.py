@@ -40,6 +40,7 @@ METRIC = "vision attn TFLOP/s & % bf16 tensor peak; ms per 50-layer tower @16384
 WORKLOAD = "tower16k: 50-layer ViT-G/14 vision-tower attention, 128x128 patches = 16384 tok, H=16, D=96"
 GRID = 128
 SCALE = 1.0 / math.sqrt(workloads.HEAD_DIM)
+INLINE_SEGMENTS = 32  # the bf16 kernel builds the work list of calls this small itself
 KERNEL_SRC = os.path.join(ROOT, "flash_attention_varlen_b200", "csrc", "attn_bf16_sm100.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_bf16_traffic.json")
 
@@ -310,6 +311,19 @@ def run_ours(args):
     ms_per_step = total_ms / args.steps
     value = step_flops * args.steps * world / (total_ms * 1e-3) / 1e12
 
+    # SM cycles per key-tile period of the busiest CTA (two 128-row Q tiles against one
+    # 128-key tile): a guard on the kernel's per-clock speed that the power-capped clock
+    # does not move (a build whose hot loop is laid out worse shows up here)
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sm_mhz = clock_info.get("sm_mhz") if isinstance(clock_info, dict) else None
+
+    def cycles_per_period(case, ms):
+        lengths = np.diff(case.cu_seqlens)
+        units = int(sum(-(-int(n) // 256) for n in lengths if n > 0)) * H
+        per_cta = -(-units // min(units, num_sms))
+        periods = per_cta * -(-int(lengths.max()) // 128)
+        return round(ms * 1e-3 * sm_mhz * 1e6 / periods) if sm_mhz else None
+
     full_traffic, win_traffic = traffic_per_launch()
     traffic = None
     if full_traffic is not None and win_traffic is not None:
@@ -349,9 +363,11 @@ def run_ours(args):
         "pct_of_bf16_peak": round(100.0 * achieved / peak, 2),
         "layers": {
             "full_16384": {"ms": round(full_ms, 4),
-                           "tflops": round(layer_flops[full_idx[0]] / (full_ms * 1e-3) / 1e12, 2)},
+                           "tflops": round(layer_flops[full_idx[0]] / (full_ms * 1e-3) / 1e12, 2),
+                           "sm_cycles_per_key_tile_period": cycles_per_period(cases[full_idx[0]], full_ms)},
             "window_16x1024": {"ms": round(win_ms, 4),
-                               "tflops": round(layer_flops[win_idx[0]] / (win_ms * 1e-3) / 1e12, 2)},
+                               "tflops": round(layer_flops[win_idx[0]] / (win_ms * 1e-3) / 1e12, 2),
+                               "sm_cycles_per_key_tile_period": cycles_per_period(cases[win_idx[0]], win_ms)},
         },
         "roofline": {
             "bound": "tensor",
@@ -366,7 +382,8 @@ def run_ours(args):
                           "averaged FLOP-weighted over the 50 calls of a step",
         },
         "configs": configs,
-        "gpu_launches": 2 * n_layers * args.steps,
+        # one launch per call; a call of more than 32 segments adds the scheduling prepass
+        "gpu_launches": args.steps * sum(1 if c.num_segments <= INLINE_SEGMENTS else 2 for c in cases),
         "e2e": e2e,
         "clocks": clock_info,
     }
