@@ -138,8 +138,11 @@ struct Smem {
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
 
 struct Unit {
-  int head, q0, seg_start, seg_end, nkv;
+  int head, q0, seg_start, seg_end;
+  int kv0, nkv;  // key tiles [kv0, kv0 + nkv) of the segment
   bool has_q1;
+  int parts, split;  // split-key units: the unit's share (split of parts) of the key tiles
+  uint32_t slot;     // split-key units: (entry, head) index, for the partial results
 };
 
 // Walks this CTA's units (one per 256 query rows of one segment and head).  The units are
@@ -159,12 +162,21 @@ struct Unit {
 // work instead of stalling every role at each unit boundary.  With a shared-memory work
 // table (a call of few segments) the entry is looked up there instead.  The unit count
 // stays below 2^31 (tokens x heads in device memory).
+//
+// In the split-key instantiation, when the call's (entry, head) units fit the workspace
+// (`split`: at most half as many as SMs), each becomes two units that take the first and
+// the second half of the segment's key tiles; the two halves are combined in the
+// epilogue.  A segment of fewer than kSplitMinKeyTiles key tiles is not split (the
+// combine costs more than half its keys save): its second unit is empty and skipped by
+// every role alike.
+template <bool kSplit>
 class UnitStream {
  public:
   __device__ __forceinline__ UnitStream(const WorkEntry* entries, const SchedTable* tab,
-                                        uint32_t E, uint32_t total, uint32_t H, int order)
+                                        uint32_t E, uint32_t total, uint32_t H, int order,
+                                        bool split = false)
       : entries_(reinterpret_cast<const int4*>(entries)), tab_(tab), E_(E), H_(H),
-        total_(total), entry_major_(order != 0) {
+        total_(total), entry_major_(order != 0), split_on_(kSplit && split) {
     locate();
   }
   __device__ __forceinline__ bool valid() const { return u_ < total_; }
@@ -175,7 +187,20 @@ class UnitStream {
     x.seg_end = cur_.w;
     x.q0 = x.seg_start + cur_.y * (2 * kBM);
     x.has_q1 = x.q0 + kBM < x.seg_end;
-    x.nkv = (x.seg_end - x.seg_start + kBN - 1) / kBN;
+    const int nkv = (x.seg_end - x.seg_start + kBN - 1) / kBN;
+    if (split_on_ && nkv >= kSplitMinKeyTiles) {
+      const int first = (nkv + 1) / 2;
+      x.parts = 2;
+      x.split = static_cast<int>(split_);
+      x.kv0 = split_ ? first : 0;
+      x.nkv = split_ ? nkv - first : first;
+    } else {
+      x.parts = 1;
+      x.split = 0;
+      x.kv0 = 0;
+      x.nkv = nkv;
+    }
+    x.slot = base_;
     ++k_;
     locate();
     return x;
@@ -184,15 +209,26 @@ class UnitStream {
  private:
   __device__ __forceinline__ void locate() {
     const uint32_t c = blockIdx.x, G = gridDim.x;
-    u_ = k_ * G + ((k_ & 1) ? G - 1 - c : c);
-    if (u_ >= total_) return;
+#pragma unroll 1
+    for (;;) {
+      u_ = k_ * G + ((k_ & 1) ? G - 1 - c : c);
+      if (u_ >= total_) return;
+      find();
+      // the second half of a segment too short to split is empty: skip it
+      if (!split_on_ || split_ == 0 || cur_.w - cur_.z > (kSplitMinKeyTiles - 1) * kBN) return;
+      ++k_;
+    }
+  }
+  __device__ __forceinline__ void find() {
+    base_ = split_on_ ? u_ >> 1 : u_;
+    split_ = split_on_ ? u_ & 1u : 0u;
     uint32_t e;
     if (entry_major_) {
-      e = u_ / H_;
-      head_ = u_ - e * H_;
+      e = base_ / H_;
+      head_ = base_ - e * H_;
     } else {
-      head_ = u_ / E_;
-      e = u_ - head_ * E_;
+      head_ = base_ / E_;
+      e = base_ - head_ * E_;
     }
     if (tab_ != nullptr) {  // the last segment whose first entry is <= e
       int s = 0;
@@ -206,8 +242,9 @@ class UnitStream {
   }
   const int4* entries_;
   const SchedTable* tab_;
-  uint32_t E_, H_, total_, k_ = 0, u_ = 0, head_ = 0;
+  uint32_t E_, H_, total_, k_ = 0, u_ = 0, head_ = 0, base_ = 0, split_ = 0;
   bool entry_major_;
+  bool split_on_;
   int4 cur_ = make_int4(0, 0, 0, 0);
 };
 
@@ -343,9 +380,10 @@ __device__ __forceinline__ void build_sched_table(SchedTable& t, const int32_t* 
 // The MMA issuer (one thread).  It is kept out of line so that its loop is one compact
 // piece of code: the thread sleeps in mbarrier waits between short bursts of MMA
 // issue, and its wake-up latency is on the critical path of every key tile.
+template <bool kSplit>
 __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem, const SchedTable* tab,
-                                      uint32_t E, uint32_t total, int order, volatile int* abort_flag,
-                                      int* dev_status) {
+                                      uint32_t E, uint32_t total, int order, bool split,
+                                      volatile int* abort_flag, int* dev_status) {
   if (a.stall_test_cycles > 0) {
     // Failure-path self-test: this wait can never succeed, so it runs out after
     // stall_test_cycles, raises the CTA's abort flag and records a timeout; every other
@@ -379,7 +417,7 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
   // where tile j+1 after a unit's last tile is the next unit's first.  So a Q tile's next S
   // is computed right after its own last PV of a unit (during that tile's epilogue), not
   // behind the other tile's last PV.  The K/V ring runs on across units as the loader fills it.
-  UnitStream us(a.entries, tab, E, total, a.H, order);
+  UnitStream<kSplit> us(a.entries, tab, E, total, a.H, order, split);
   bool ok = us.valid();
   Unit x;
   if (ok) {
@@ -457,14 +495,20 @@ __device__ __noinline__ void mma_role(Smem& sm, const Bf16Args& a, uint32_t tmem
   mbar_wait_drain(&sm.drain, 0);
 }
 
-// kStageO: whole O tiles leave through the Q buffers and TMA stores (warp 11), else every
-// row is stored by its thread and warp 11 idles.  Two instantiations, because the staging
-// code alone, never run, moved the softmax loop's code enough to cost ~1.5% on long units.
-template <bool kStageO>
+// The epilogue, fixed per instantiation:
+//   kEpiRows   every row is stored by its thread; warp 11 idles;
+//   kEpiStaged whole O tiles leave through the Q buffers and TMA stores (warp 11);
+//   kEpiSplit  the split-key units: each half writes its unnormalised rows with (m, l) to
+//              a workspace and the second half to finish combines the two.
+// Separate instantiations, because the staging code alone, never run, moved the softmax
+// loop's code enough to cost ~1.5% on long units.
+template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
                      const __grid_constant__ Bf16Args a) {
+  constexpr bool kStageO = kEpi == kEpiStaged;
+  constexpr bool kSplit = kEpi == kEpiSplit;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (raw & 1023u)) & 1023u));
@@ -547,7 +591,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     E = static_cast<uint32_t>(a.hdr->num_entries);
     order = a.hdr->order;
   }
-  const uint32_t total = E * static_cast<uint32_t>(a.H);
+  // split-key units when this call's (entry, head) units fit the workspace: decided here,
+  // from the work list itself, so the in-kernel and prepass work lists split alike
+  const bool split = kSplit && E * static_cast<uint32_t>(a.H) <= static_cast<uint32_t>(a.split_units_max);
+  const uint32_t total = E * static_cast<uint32_t>(a.H) * (split ? 2u : 1u);
   if (blockIdx.x >= total) {  // uniform over the CTA: no unit for it
     if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
     return;
@@ -560,12 +607,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kv_it = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
-      for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid() && ok;) {
+      for (UnitStream<kSplit> us(a.entries, tab, E, total, a.H, order, split); us.valid() && ok;) {
         const Unit x = us.take();
         for (int j = 0; j < x.nkv; ++j, ++kv_it) {
           const uint32_t sk = kv_it % kKStages, fk = kv_it / kKStages;
           const uint32_t sv = kv_it % kVStages, fv = kv_it / kVStages;
-          const int row0 = x.seg_start + j * kBN;
+          const int row0 = x.seg_start + (x.kv0 + j) * kBN;
           if (fk > 0 && !mbar_wait_bounded(&sm.k_empty[sk], (fk - 1) & 1, abort_flag, dev_status)) {
             ok = false;
             break;
@@ -599,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // per-buffer load counts (kept in scalars: a runtime-indexed array would go to local memory)
       uint32_t unit_it = 0, q0a = 0, q0b = 0, q1a = 0, q1b = 0;
-      for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid(); ++unit_it) {
+      for (UnitStream<kSplit> us(a.entries, tab, E, total, a.H, order, split); us.valid(); ++unit_it) {
         const Unit x = us.take();
         const uint32_t b = unit_it % kQBufs, use = unit_it / kQBufs;
         // buffer b is free once every QK of the unit that used it before has completed and
@@ -628,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
    } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      mma_role(sm, a, tmem, tab, E, total, order, abort_flag, dev_status);
+      mma_role<kSplit>(sm, a, tmem, tab, E, total, order, split, abort_flag, dev_status);
     }
    } else if (kStageO && warp == kWarpStore) {
     // ------------------------------------------------------------ O tile stores
@@ -641,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t unit_it = 0, staged = 0;  // bit 2b + i: parity of (buffer b, tile i) stagings
       bool ok = true;
-      for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid() && ok; ++unit_it) {
+      for (UnitStream<kSplit> us(a.entries, tab, E, total, a.H, order, split); us.valid() && ok; ++unit_it) {
         const Unit x = us.take();
         const uint32_t b = unit_it % kQBufs;
         if (!mbar_wait_bounded(&sm.q_full[b][0], (unit_it / kQBufs) & 1, abort_flag, dev_status)) break;
@@ -683,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + (wg ? kColO1 : kColO0);
     const float c = a.scale_log2;
     uint32_t s_cnt = 0, o_base = 0, unit_it = 0;
-    for (UnitStream us(a.entries, tab, E, total, a.H, order); us.valid();) {
+    for (UnitStream<kSplit> us(a.entries, tab, E, total, a.H, order, split); us.valid();) {
       const Unit x = us.take();
       const uint32_t b = unit_it++ % kQBufs;
       if (wg == 1 && !x.has_q1) continue;
@@ -694,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!warp_wait(&sm.s_full[wg], s_cnt & 1, abort_flag, dev_status)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
-        const int nvalid = x.seg_end - (x.seg_start + j * kBN);  // >= 1
+        const int nvalid = x.seg_end - (x.seg_start + (x.kv0 + j) * kBN);  // >= 1
         const bool masked = nvalid < kBN;
         float pm[8];
         // pass 1, row max: the row in two 64-column halves, eight independent
@@ -811,7 +858,63 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       reg_fence<kD + 1>(o);
       const bool whole = kStageO && x.q0 + wg * kBM + kBM <= x.seg_end;  // staged for a TMA store
-      if (whole || row_tok < x.seg_end) {
+      if (kSplit && x.parts == 2) {
+        // A split-key unit holds O and l over its half of the keys, both relative to
+        // 2^m.  Each half writes its tile (per row: 96 values, m, l) as 25 float4 columns
+        // of 128 rows, so a warp stores 512 contiguous bytes at a time.  Then, per warp,
+        // lane 0 swaps this call's id into the warp's flag (release: the warp's rows are
+        // visible first); the half that finds the id there finished second (acquire: the
+        // other half's rows are visible) and combines the two into O.  The warp-uniform
+        // flow keeps the shuffles and __syncwarp convergent.
+        const size_t tile_id = static_cast<size_t>(x.slot) * 2 + wg;
+        float4* mine = reinterpret_cast<float4*>(a.part) + (tile_id * 2 + x.split) * (kPartF4 * kBM) + r;
+        const float4* other =
+            reinterpret_cast<const float4*>(a.part) + (tile_id * 2 + (x.split ^ 1)) * (kPartF4 * kBM) + r;
+        const float l_own = __uint_as_float(o[96]);
+#pragma unroll
+        for (int i = 0; i < kD / 4; ++i)
+          __stcg(mine + i * kBM,
+                 make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                             __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3])));
+        __stcg(mine + (kD / 4) * kBM, make_float4(m, l_own, 0.f, 0.f));
+        __syncwarp();
+        uint32_t seen = 0;
+        if (lane == 0) seen = atom_exch_acq_rel_gpu(a.part_flag + tile_id * 4 + (warp & 3), a.call_id);
+        seen = __shfl_sync(0xffffffffu, seen, 0);
+        __syncwarp();  // lane 0's acquire orders the other lanes' reads below too
+        if (seen == a.call_id && row_tok < x.seg_end) {
+          // the arithmetic runs on (first half, second half) whichever half combines,
+          // so the result does not depend on which finished first
+          const bool first = x.split == 0;
+          const float4 ml = __ldcg(other + (kD / 4) * kBM);
+          const float m0 = first ? m : ml.x, m1 = first ? ml.x : m;
+          const float l0 = first ? l_own : ml.y, l1 = first ? ml.y : l_own;
+          const float mm = fmaxf(m0, m1);
+          const float a0 = exp2f(m0 - mm), a1 = exp2f(m1 - mm);
+          const float inv = 1.0f / fmaf(a0, l0, a1 * l1);
+          const float c0 = a0 * inv, c1 = a1 * inv;
+          uint32_t w[kD / 2];
+#pragma unroll
+          for (int i = 0; i < kD / 4; ++i) {
+            const float4 ov = __ldcg(other + i * kBM);
+            const float4 ow = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                          __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            const float4 h0 = first ? ow : ov, h1 = first ? ov : ow;
+            w[2 * i] = pack_bf16x2(fmaf(c0, h0.x, c1 * h1.x), fmaf(c0, h0.y, c1 * h1.y));
+            w[2 * i + 1] = pack_bf16x2(fmaf(c0, h0.z, c1 * h1.z), fmaf(c0, h0.w, c1 * h1.w));
+          }
+          uint8_t* row = static_cast<uint8_t*>(a.out) +
+                         (static_cast<size_t>(row_tok) * a.H + x.head) * (kD * 2);
+          if (a.out_align32) {
+#pragma unroll
+            for (int i = 0; i < kD / 16; ++i) st_global_v8(row + 32 * i, w + 8 * i);
+          } else {
+#pragma unroll
+            for (int i = 0; i < kD / 8; ++i)
+              reinterpret_cast<uint4*>(row)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+      } else if (whole || row_tok < x.seg_end) {
         const float inv_l = 1.0f / __uint_as_float(o[96]);
         const float2 il2 = make_float2(inv_l, inv_l);
         uint32_t w[kD / 2];
@@ -869,7 +972,7 @@ size_t bf16_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, const Bf16Args& args, int grid,
-                             bool stage_o, cudaStream_t stream) {
+                             int epilogue, cudaStream_t stream) {
   // Programmatic stream serialization: the kernel may launch while the scheduling prepass
   // before it still runs, and waits for it (griddepcontrol.wait) before reading its output.
   cudaLaunchConfig_t cfg = {};
@@ -882,16 +985,25 @@ cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return stage_o ? cudaLaunchKernelEx(&cfg, attn_bf16_kernel<true>, tq, tk, tv, to, args)
-                 : cudaLaunchKernelEx(&cfg, attn_bf16_kernel<false>, tq, tk, tv, to, args);
+  switch (epilogue) {
+    case kEpiRows: return cudaLaunchKernelEx(&cfg, attn_bf16_kernel<kEpiRows>, tq, tk, tv, to, args);
+    case kEpiStaged: return cudaLaunchKernelEx(&cfg, attn_bf16_kernel<kEpiStaged>, tq, tk, tv, to, args);
+    case kEpiSplit: return cudaLaunchKernelEx(&cfg, attn_bf16_kernel<kEpiSplit>, tq, tk, tv, to, args);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t prepare_attn_bf16() {
-  const cudaError_t e = cudaFuncSetAttribute(
-      attn_bf16_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(attn_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(kSmemBytes));
+  const int bytes = static_cast<int>(kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<kEpiRows>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bf16_kernel<kEpiStaged>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bf16_kernel<kEpiSplit>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  return e;
 }
 
 }  // namespace vt

@@ -34,9 +34,10 @@ struct alignas(16) WorkEntry {
   int32_t seg_end;    // cu_seqlens[seg + 1]
 };
 
-// Entries that a call can produce at most: sum_s ceil(L_s / rows) <= T / rows + n.
+// Entries that a call can produce at most: each ceil(L_s / R) <= (L_s + R - 1) / R, so the
+// sum is at most floor((T + n (R - 1)) / R) (exact for one segment).
 inline int64_t max_work_entries(int64_t total_tokens, int64_t num_segments, int block_rows) {
-  return (total_tokens + block_rows - 1) / block_rows + num_segments;
+  return (total_tokens + num_segments * (block_rows - 1)) / block_rows;
 }
 
 inline size_t scratch_bytes_for(int64_t total_tokens, int64_t num_segments, int block_rows) {
@@ -88,7 +89,33 @@ struct Bf16Args {
   // > 0 only in the failure-path self-test: the MMA thread first waits this many cycles
   // on a barrier that never completes (see vt_attn_selftest_wait_timeout)
   int32_t stall_test_cycles = 0;
+  // split-key epilogue only: the halves' tiles (kPartF4 float4 columns of 128 rows each;
+  // tile t's halves at 2 t and 2 t + 1), one flag per 32-row warp slice of a tile, and
+  // this call's id (never 0)
+  float* part = nullptr;
+  uint32_t* part_flag = nullptr;
+  uint32_t call_id = 0;
+  int32_t split_units_max = 0;  // the kernel splits when the call's units are at most this
 };
+// The kernel's epilogue modes (one instantiation each): per-thread row stores; whole tiles
+// staged in the Q buffers and stored by TMA; split-key units combined in the epilogue.
+constexpr int kEpiRows = 0, kEpiStaged = 1, kEpiSplit = 2;
+// Split-key units: segments of at least this many 128-key tiles are split (measured: with
+// one key tile per half the combine, ~4 us, costs more than the half it saves).
+constexpr int kSplitMinKeyTiles = 4;
+// A split-key row: 96 unnormalised O values, then (m, l, 0, 0): 25 float4.
+constexpr int kPartF4 = 25;
+// Workspace of the split-key epilogue for up to `units` (entry, head) units: the rows'
+// halves, then the flags (zeroed once when allocated; a flag holds the id of the last call
+// that wrote it, so it needs no reset between calls).
+// A unit has two 128-row tiles; tile (unit u, tile i) is 2 u + i, with two halves of
+// kPartF4 * 128 float4 each and four flags (one per warp of 32 rows).
+inline size_t split_part_bytes(long long units) {
+  return static_cast<size_t>(units) * 2 * 2 * kPartF4 * 128 * 16;
+}
+inline size_t split_flag_bytes(long long units) {
+  return static_cast<size_t>(units) * 2 * 4 * sizeof(uint32_t);
+}
 size_t bf16_smem_bytes();
 cudaError_t prepare_attn_bf16();  // opt in to the kernel's dynamic shared memory (per device)
 // `to` maps the output like tq maps Q (same shape, box and swizzle).  With stage_o, whole
@@ -96,7 +123,7 @@ cudaError_t prepare_attn_bf16();  // opt in to the kernel's dynamic shared memor
 // (worth it when a CTA runs several short units: the stores overlap the next unit);
 // otherwise every row is stored by its thread.
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& to, const Bf16Args& args, int grid, bool stage_o,
+                             const CUtensorMap& to, const Bf16Args& args, int grid, int epilogue,
                              cudaStream_t stream);
 // The staged epilogue is chosen for calls whose segments average at most this many tokens
 // and that give each SM at least kStageMinUnitsPerSm units of 256 rows on average.
@@ -151,6 +178,12 @@ struct FwdCall {
   int dtype;  // vt_dtype
   cudaStream_t stream;
   int32_t stall_test_cycles;  // > 0 only for the bf16 failure-path self-test
+  // bf16 only: a workspace for split-key units (split_part_bytes / split_flag_bytes of
+  // max_work_entries(...) * H units) and this call's id; null: no split-key units
+  float* part = nullptr;
+  uint32_t* part_flag = nullptr;
+  uint32_t call_id = 0;
+  int32_t split_units_max = 0;
 };
 
 // Host-side argument checks shared by every forward entry point; touches no device.

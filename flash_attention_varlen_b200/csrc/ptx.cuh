@@ -281,6 +281,18 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 
 // Generic-proxy writes to shared memory made visible to the async proxy
 // (tensor core / TMA) before they read it.
+// Atomic exchange with acquire-release ordering at GPU scope: this thread's earlier writes
+// are visible to whoever reads the new value, and its later reads see what the thread
+// that wrote the old value had written before its own exchange.
+__device__ __forceinline__ uint32_t atom_exch_acq_rel_gpu(uint32_t* addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.exch.b32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(addr), "r"(v)
+               : "memory");
+  return old;
+}
+
 // TMA tile store from shared memory (the same box and swizzle as the map's loads); its
 // completion is tracked per issuing thread by bulk async-groups.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int c0,

@@ -37,6 +37,11 @@ struct Scratch {
   size_t bytes = 0;
   uint32_t calls = 0;  // forward calls queued on this scratch: their status slots alternate
   int last_slot = 0;   // status slot of the latest one
+  // the split-key epilogue's workspace (rows' halves, then per-row flags) for up to
+  // split_units units, and the id of the latest call that used it
+  void* split_ptr = nullptr;
+  long long split_units = 0;
+  uint32_t split_calls = 0;
 };
 
 std::mutex g_mu;      // the per-stream work lists
@@ -233,7 +238,13 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) 
     a.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(c.scale)) * log2e);
     a.idesc_qk = make_idesc_bf16(128, 128, false, false, c.scale < 0.0f);
     a.stall_test_cycles = c.stall_test_cycles;
-    const int grid = static_cast<int>(max_units < di->num_sms ? max_units : di->num_sms);
+    const bool split = c.part != nullptr;
+    a.part = c.part;
+    a.part_flag = c.part_flag;
+    a.call_id = c.call_id;
+    a.split_units_max = c.split_units_max;
+    const long long units = split ? 2 * max_units : max_units;
+    const int grid = static_cast<int>(units < di->num_sms ? units : di->num_sms);
     // Staged O stores pay off when a CTA runs several short units (window layers); with
     // one or two units per CTA the store's tail latency costs more than it hides.  The
     // host sees only T and n (cu_seqlens stays on the device), so the rule uses the mean.
@@ -241,7 +252,8 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) 
     const bool stage_o =
         static_cast<int64_t>(c.total_tokens) <= static_cast<int64_t>(kStageMaxMeanSegment) * c.num_segments &&
         rows_x_heads >= static_cast<int64_t>(kStageMinUnitsPerSm) * di->num_sms * kBf16BlockRows;
-    if (launch_attn_bf16(tq, tk, tv, to, a, grid, stage_o, c.stream) != cudaSuccess) return VT_ERR_CUDA;
+    const int epilogue = split ? kEpiSplit : stage_o ? kEpiStaged : kEpiRows;
+    if (launch_attn_bf16(tq, tk, tv, to, a, grid, epilogue, c.stream) != cudaSuccess) return VT_ERR_CUDA;
   } else {
     F32Args a;
     a.q = static_cast<const float*>(c.q);
@@ -264,6 +276,8 @@ int launch_fwd(const FwdCall& c, WorkHeader* hdr, WorkEntry* entries, int slot) 
 
 namespace {
 
+int sm_count();  // of the current device; 0 if it cannot be read
+
 // The forward of a validated call with the library-owned, per-(device, stream) work list.
 vt_status fwd_impl(const vt::FwdCall& c) {
   int dev = 0;
@@ -276,10 +290,46 @@ vt_status fwd_impl(const vt::FwdCall& c) {
                    &sc);
   if (st != VT_OK) return st;
   auto* hdr = static_cast<vt::WorkHeader*>(sc->ptr);
+  vt::FwdCall call = c;
+  // A bf16 call with at most half as many (entry, head) units as SMs splits each unit's
+  // keys over two CTAs (two units) and combines them in the kernel's epilogue.  The kernel
+  // counts the units from the work list and decides; the host only rules the split out
+  // when even the fewest units the call can have, ceil(T / 256) per head, are too many,
+  // or when no segment can be long enough to split.
+  const long long fewest =
+      (static_cast<long long>(c.total_tokens) + vt::kBf16BlockRows - 1) / vt::kBf16BlockRows * c.H;
+  const int nsm = sm_count();
+  if (c.dtype == VT_DTYPE_BF16 && nsm > 1 && 2 * fewest <= nsm &&
+      c.total_tokens > (vt::kSplitMinKeyTiles - 1) * 128) {
+    if (sc->split_units < nsm / 2) {
+      if (sc->split_ptr) {
+        if (cudaStreamSynchronize(c.stream) != cudaSuccess) return VT_ERR_CUDA;
+        cudaFree(sc->split_ptr);
+        sc->split_ptr = nullptr;
+        sc->split_units = 0;
+      }
+      const long long cap = nsm / 2;  // covers every call that can split on this device
+      const size_t part = vt::split_part_bytes(cap), flags = vt::split_flag_bytes(cap);
+      if (cudaMalloc(&sc->split_ptr, part + flags) != cudaSuccess) {
+        sc->split_ptr = nullptr;
+        return VT_ERR_CUDA;
+      }
+      if (cudaMemsetAsync(static_cast<char*>(sc->split_ptr) + part, 0, flags, c.stream) !=
+          cudaSuccess)
+        return VT_ERR_CUDA;
+      sc->split_units = cap;
+    }
+    if (++sc->split_calls == 0) sc->split_calls = 1;  // 0 is the flags' initial value
+    call.part = static_cast<float*>(sc->split_ptr);
+    call.part_flag = reinterpret_cast<uint32_t*>(static_cast<char*>(sc->split_ptr) +
+                                                 vt::split_part_bytes(sc->split_units));
+    call.call_id = sc->split_calls;
+    call.split_units_max = static_cast<int32_t>(sc->split_units);
+  }
   const int slot = static_cast<int>(sc->calls++ & 1u);
   sc->last_slot = slot;
   return static_cast<vt_status>(
-      vt::launch_fwd(c, hdr, reinterpret_cast<vt::WorkEntry*>(hdr + 1), slot));
+      vt::launch_fwd(call, hdr, reinterpret_cast<vt::WorkEntry*>(hdr + 1), slot));
 }
 
 // The text decoder's attention: validated arguments, the prepass (128-row entries) and the

@@ -21,8 +21,11 @@
  * (device, stream), one small scratch buffer for its work list: it is
  * allocated on the first call on that stream and grown (never shrunk) when a
  * call needs more; make a first call on a stream before capturing it in a
- * CUDA graph.  Calls are stream-ordered; calls on different streams use
- * different scratch buffers.  The library keeps per-device state (launch
+ * CUDA graph.  A bf16 call with at most half as many (256-row block, head) units as
+ * the device has SMs splits each unit's keys over two CTAs and combines the halves in
+ * the kernel; its first such call on a stream also allocates, once, a workspace for
+ * the halves (about 100 KB per SM).  Calls are stream-ordered; calls on different
+ * streams use different scratch buffers.  The library keeps per-device state (launch
  * attributes, work lists, device addresses) for the life of the device's primary
  * context: a cudaDeviceReset invalidates it, so do not call the library again in a
  * process after resetting a device it has used.
@@ -94,14 +97,17 @@ vt_status vt_attn_fwd(const void* q, const void* k, const void* v, void* out,
  * process exits) instead of a per-stream allocation.
  *
  * Limits and rules:
- *   - the work list must fit: 128 + 16 * (ceil(T / R) + num_segments) <= 1 MiB,
- *     R = 256 for bf16, 64 for f32 (e.g. bf16 T = 16384 with 16 segments uses
- *     1408 bytes); larger calls return VT_ERR_UNSUPPORTED and launch nothing;
+ *   - the work list must fit: 128 + 16 * floor((T + num_segments * (R - 1)) / R)
+ *     <= 1 MiB, R = 256 for bf16, 128 for f32 (e.g. bf16 T = 16384 with 16 segments
+ *     uses 1392 bytes); larger calls return VT_ERR_UNSUPPORTED and launch nothing;
  *   - the first call on a device looks up the array's device address for that
  *     device (make it with the device current, before capturing the stream into
  *     anything);
  *   - every call on a device shares the array, so calls that may overlap on the
  *     GPU (e.g. on two streams) race and must be serialised by the caller;
+ *   - it never splits a unit's keys over two CTAs (its array has no room for that
+ *     workspace), so on calls small enough for vt_attn_fwd to do so (at most half as
+ *     many (256-row block, head) units as SMs) the two differ in rounding;
  *   - what the device side finds is not reported: vt_attn_last_device_status covers
  *     vt_attn_fwd's own work lists only.  A malformed cu_seqlens makes the call write
  *     nothing; a kernel wait that gives up (VT_ERR_DEVICE_TIMEOUT for vt_attn_fwd, a

@@ -76,9 +76,10 @@ def test_smem_contract(binding):
 
 
 def test_workspace_bytes(binding):
-    # header (128 B) + 16 B per entry, entries <= ceil(T / rows) + n
-    assert binding.vt_attn_workspace_bytes(16, 16384, binding.VT_DTYPE_BF16) == 128 + 16 * (64 + 16)
-    assert binding.vt_attn_workspace_bytes(1, 256, binding.VT_DTYPE_F32) == 128 + 16 * (2 + 1)
+    # header (128 B) + 16 B per entry; entries = sum_s ceil(L_s / rows) <= floor((T + n (rows - 1)) / rows)
+    assert binding.vt_attn_workspace_bytes(16, 16384, binding.VT_DTYPE_BF16) == 128 + 16 * ((16384 + 16 * 255) // 256)
+    assert binding.vt_attn_workspace_bytes(1, 256, binding.VT_DTYPE_F32) == 128 + 16 * 2
+    assert binding.vt_attn_workspace_bytes(1, 1024, binding.VT_DTYPE_BF16) == 128 + 16 * 4
     assert binding.vt_attn_workspace_bytes(-1, 5, binding.VT_DTYPE_BF16) == 0
 
 

@@ -324,7 +324,10 @@ def _round_bf16(x):
 
 
 def test_block_diagonal_independence_and_packing_order_bitwise():
-    lens = [300, 1024, 77, 513]
+    # each segment alone still makes 80 (256-row block, head) units, more than half the
+    # SMs, so no call here splits its units' keys (a split call sums a row's keys in two
+    # halves: see test_split_key_units); ragged ends 76, 20 and 16 rows into a tile
+    lens = [1100, 1300, 1040, 1280]
     cu = workloads.cu_from_lengths(lens)
     case = workloads.Case("indep", cu, seed=9, dtype="bf16")
     q, k, v = case.inputs()
@@ -338,6 +341,40 @@ def test_block_diagonal_independence_and_packing_order_bitwise():
     cu2 = workloads.cu_from_lengths([lens[s] for s in order])
     out2 = _run(perm(q), perm(k), perm(v), cu2, "bf16")
     assert np.array_equal(out2, perm(batch))
+
+
+def test_split_key_units():
+    """Calls with at most half as many (256-row block, head) units as SMs split each unit's
+    key tiles over two CTAs and combine the halves in the epilogue (segments of at least 4
+    key tiles).  Segments of 1, 2, 3 (not split), 6 and 9 key tiles, a negative scale,
+    every element against the oracle; the
+    same call again is bit-identical (the combine does not depend on which half finishes
+    first); and a segment computed split (alone) and unsplit (inside a batch too large to
+    split) both meet the bound against the oracle and differ only by rounding: each
+    rounds P to bf16 against its own running max, so they disagree by about the kernel's
+    own error (mean-abs ~1e-4), not by a whole value."""
+    lengths = [129, 300, 1, 700, 77, 1100]
+    cu = workloads.cu_from_lengths(lengths)
+    case = workloads.Case("split_keys", cu, seed=13, dtype="bf16", H=4)
+    q, k, v = case.inputs()
+    ref = oracle.attn_fwd(q, k, v, cu, -0.3)
+    got = _run(q, k, v, cu, "bf16", scale=-0.3)
+    _check(got, ref, "bf16", "split-key units")
+    assert np.array_equal(got, _run(q, k, v, cu, "bf16", scale=-0.3))
+    # the 700-token segment alone (split) against the same rows in a 16-head batch of 9000
+    # tokens (not split)
+    big = workloads.Case("no_split", workloads.cu_from_lengths([700] + [1100] * 7 + [600]), seed=14,
+                         dtype="bf16")
+    bq, bk, bv = big.inputs()
+    seg = np.array([0, 700], np.int32)
+    batch = _run(bq, bk, bv, big.cu_seqlens, "bf16")[:700]
+    alone = _run(bq[:700], bk[:700], bv[:700], seg, "bf16")
+    ref700 = oracle.attn_fwd(bq[:700], bk[:700], bv[:700], seg, SCALE)
+    _check(alone, ref700, "bf16", "700 tokens alone (split)")
+    _check(batch, ref700, "bf16", "700 tokens in the batch (unsplit)")
+    diff = np.abs(alone - batch)
+    assert diff.mean() <= 3e-4 and diff.max() <= 5e-3, (diff.mean(), diff.max())
+    assert not np.array_equal(alone, batch)  # the two really are different summation orders
 
 
 def test_deterministic():

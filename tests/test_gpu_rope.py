@@ -70,6 +70,24 @@ def test_rope2d_matches_oracle_on_the_tower_grid(theta):
     assert np.mean(np.abs(got - ref)) <= 1.01 * np.mean(np.abs(ref_bf16 - ref))
 
 
+def test_rope2d_odd_head_count_and_more_items_than_threads():
+    """H = 9 (rows of a token not a multiple of any block) and 40,000 tokens: 2.16M
+    (token, head, group) items against a grid of at most 148 x 64 blocks of 192 threads
+    (1.82M), so threads take a second item on the grid stride, each staying on its own
+    column group.  Every element within the one-ulp bound of the oracle."""
+    import flash_attention_varlen_b200 as fa
+    T, H = 40000, 9
+    q, _, _ = workloads.qkv(39, T, H=H)
+    pos = np.random.default_rng(6).integers(1, 400, size=(T, 2)).astype(np.int32)
+    got = fa.rope2d(_bf16_dev(q), torch.from_numpy(pos).cuda())
+    torch.cuda.synchronize()
+    got = got.float().cpu().numpy().astype(np.float64)
+    ref = rope.rope2d(q, pos)
+    ang = rope.rope_angles(pos, 96, rope.DEFAULT_THETA)
+    ok = _within_one_ulp(got, ref, workloads.bf16_bits_to_f32(q).astype(np.float64), ang)
+    assert np.isfinite(got).all() and ok.all(), f"{(~ok).sum()} elements beyond one ulp"
+
+
 def test_rope2d_in_place_equals_out_of_place_and_position_zero_is_identity():
     import flash_attention_varlen_b200 as fa
     T, H = 300, 3

@@ -64,6 +64,8 @@ def _check_close(got, ref, dtype):
 
 
 def _cases():
+    # all too large for vt_attn_fwd's split-key units (which the no-alloc entry point never
+    # uses), so the two run the same kernel on the same work list
     return [workloads.varlen8_case(),
             workloads.Case("ragged_f32", workloads.cu_from_lengths([1, 127, 0, 129, 300, 64]),
                            seed=11, dtype="f32"),
@@ -120,7 +122,7 @@ def test_noalloc_allocates_nothing_on_a_fresh_stream():
 
 def test_noalloc_rejects_work_lists_beyond_its_array():
     from flash_attention_varlen_b200 import _binding as b
-    # 200000 one-token segments need 128 + 16 * (782 + 200000) bytes > 1 MiB: refused on the
+    # 200000 one-token segments need 128 + 16 * 200000 bytes > 1 MiB: refused on the
     # host before anything is launched (the pointers below are never dereferenced).
     T = n = 200000
     cu = np.zeros(4, np.int32)
