@@ -35,6 +35,10 @@
 //                        128-row tile is staged in the unit's Q buffer (its QKs are
 //                        done) and warp 11 sends it out with TMA stores, while the
 //                        rows of a tile cut by its segment's end still go row by row.
+//                        In the split-key instantiation (calls of at most half as
+//                        many units as SMs) a unit may take half of its segment's key
+//                        tiles; its rows are combined with the other half's through
+//                        a workspace in global memory (see the epilogue).
 //
 // CTAs take their units in a longest-first snake order (see UnitStream).
 //
