@@ -59,7 +59,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time budget of the oracle sample")
     ap.add_argument("--single-layer", choices=["full", "window", "varlen8", "f32_4096",
-                                               "decoder_sliding", "decoder_full"], default=None,
+                                               "decoder_sliding", "decoder_full", "rope2d_window"],
+                    default=None,
                     help="profiling aid: run only one layer (full = 1 x 16384 tok, window = "
                          "16 x 1024 tok, varlen8 = eight images of unequal size) warmup + "
                          "steps times and print its timing")
@@ -761,8 +762,9 @@ def run_reference(args):
 
 def run_single_layer(args):
     """One layer, called warmup + steps times (for ncu captures): a tower layer type, the
-    eight-image batch, a 4096-token f32 segment (the f32 arm) or the text decoder's sliding
-    or full layer on a 16384-token sequence."""
+    eight-image batch, a 4096-token f32 segment (the f32 arm), the text decoder's sliding
+    or full layer on a 16384-token sequence, or the tower's window layer with the 2D RoPE
+    (the rotation pass over Q and K, then the attention)."""
     import torch
     import flash_attention_varlen_b200 as fa
     dev = torch.device("cuda", 0)
@@ -790,6 +792,11 @@ def run_single_layer(args):
         cu = torch.from_numpy(case.cu_seqlens.copy()).to(dev)
         out = torch.empty_like(dq)
         call = lambda: fa.attn_fwd(dq, dk, dv, cu, scale=SCALE, out=out)
+        if args.single_layer == "rope2d_window":
+            perm, _ = fa.window_partition([(GRID, GRID)], 32, device=dev)
+            pos = torch.from_numpy(workloads.patch_positions(GRID, GRID)).to(dev)[perm.long()].contiguous()
+            k_rot = torch.empty_like(dk)
+            call = lambda: fa.attn_fwd_rope2d(dq, dk, dv, cu, pos, scale=SCALE, out=out, k_rot=k_rot)
     for _ in range(args.warmup):
         call()
     fa.check_device_status()
