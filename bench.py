@@ -319,10 +319,7 @@ def run_ours(args):
     sm_mhz = clock_info.get("sm_mhz") if isinstance(clock_info, dict) else None
 
     def cycles_per_period(case, ms):
-        lengths = np.diff(case.cu_seqlens)
-        units = int(sum(-(-int(n) // 256) for n in lengths if n > 0)) * H
-        per_cta = -(-units // min(units, num_sms))
-        periods = per_cta * -(-int(lengths.max()) // 128)
+        periods = key_tile_periods(case.cu_seqlens, H, num_sms)
         return round(ms * 1e-3 * sm_mhz * 1e6 / periods) if sm_mhz else None
 
     full_traffic, win_traffic = traffic_per_launch()
@@ -398,6 +395,16 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def key_tile_periods(cu_seqlens, H: int, num_sms: int) -> int:
+    """Key-tile periods of the busiest CTA of a bf16 call with equal-cost units: units of
+    256 query rows per (segment, head), dealt over min(units, SMs) persistent CTAs, each
+    unit taking one period per 128-key tile of its segment (the longest segment's count)."""
+    lengths = np.diff(np.asarray(cu_seqlens, np.int64))
+    units = int(sum(-(-int(n) // 256) for n in lengths if n > 0)) * H
+    per_cta = -(-units // min(units, num_sms))
+    return per_cta * -(-int(lengths.max()) // 128)
 
 
 def config_cases():

@@ -59,3 +59,17 @@ def test_gpus_flag_must_match_the_launched_ranks(monkeypatch, capsys):
     assert e.value.code == 2 and "--gpus 8" in capsys.readouterr().err
     monkeypatch.setenv("WORLD_SIZE", "4")
     bench.check_world(bench.parse_args(["--gpus", "4"]))
+
+
+def test_key_tile_periods_of_the_tower_layers():
+    """The per-clock guard's denominator: on 148 SMs the full layer (1 x 16384 tokens, 16
+    heads) makes 1024 units of 128 key tiles, 7 on the busiest CTA; the window layer (16 x
+    1024) makes 1024 units of 8 key tiles, also 7 per CTA."""
+    import bench
+    import workloads
+    full = workloads.cu_from_lengths([16384])
+    window = workloads.cu_from_lengths([1024] * 16)
+    assert bench.key_tile_periods(full, 16, 148) == 7 * 128
+    assert bench.key_tile_periods(window, 16, 148) == 7 * 8
+    # fewer units than SMs: one unit per CTA
+    assert bench.key_tile_periods(workloads.cu_from_lengths([1024]), 16, 148) == 8
