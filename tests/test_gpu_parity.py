@@ -176,6 +176,23 @@ def test_staged_output_tiles_with_ragged_segment_ends():
     _full_case(case)
 
 
+def test_staged_epilogue_many_short_units_through_the_prepass():
+    """600 segments of 128, 200, 256, 300 and 77 tokens over 4 heads: the staged epilogue
+    (mean length 192, many units per SM) with ~16 short units per CTA, so the Q buffers
+    are released to the loader after each unit's TMA stores every few thousand cycles;
+    more than 32 segments, so the work list comes from the prepass.  Whole 128-row tiles
+    go through the stores, the 72-, 44- and 77-row remainders row by row.  One row in every
+    (256-row entry, head) unit against the oracle."""
+    lengths = [128, 200, 256, 300, 77] * 120
+    cu = workloads.cu_from_lengths(lengths)
+    case = workloads.Case("staged_short_units", cu, seed=15, dtype="bf16", H=4)
+    q, k, v = case.inputs()
+    got = _run(q, k, v, cu, "bf16")
+    tok, head = _unit_rows(cu, 4, 15)
+    ref = oracle.attn_rows(q, k, v, cu, SCALE, tok, head)
+    _check(got[tok, head], ref, "bf16", case.name)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_more_segments_than_the_prepass_sorts(dtype):
     # 5000 segments (the prepass sorts at most 4096: more keep their given order and
