@@ -58,7 +58,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time budget of the oracle sample")
-    ap.add_argument("--single-layer", choices=["full", "window", "varlen8", "f32_4096",
+    ap.add_argument("--single-layer", choices=["full", "window", "varlen8", "f32_4096", "img448",
                                                "decoder_sliding", "decoder_full", "rope2d_window"],
                     default=None,
                     help="profiling aid: run only one layer (full = 1 x 16384 tok, window = "
@@ -788,6 +788,8 @@ def run_single_layer(args):
     else:
         if args.single_layer == "varlen8":  # eight images of unequal size (the scheduler's case)
             case = workloads.varlen8_case(0)
+        elif args.single_layer == "img448":  # one 448 x 448 image: split-key units
+            case = workloads.image448_case()
         elif args.single_layer == "f32_4096":
             case = workloads.Case("f32_4096", workloads.cu_from_lengths([4096]), seed=5, dtype="f32")
         else:
