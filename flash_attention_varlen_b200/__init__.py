@@ -30,7 +30,7 @@ __all__ = ["attn_fwd", "attn_fwd_swa", "attn_fwd_host", "window_partition", "per
            "rope2d", "attn_fwd_rope2d",
            "check_device_status", "VtAttnError", "vt_attn_fwd",
            "vt_attn_validate_seqlens_host", "vt_attn_smem_bytes", "vt_attn_workspace_bytes",
-           "vt_attn_last_device_status", "status_string", "vt_attn_version"]
+           "vt_attn_last_device_status", "status_string", "vt_attn_version", "set_split_keys"]
 
 
 def _dtype_code(t):
@@ -122,6 +122,13 @@ def attn_fwd_swa(q, k, v, cu_seqlens, window: int = 0, scale: float | None = Non
     if rc != VT_OK:
         raise VtAttnError(rc, "vt_attn_fwd_swa")
     return out
+
+
+def set_split_keys(enable: bool) -> bool:
+    """Allow (True, the default) or forbid splitting a unit's keys over two CTAs in small
+    bf16 calls.  Forbidding it makes a segment's output the same bits whatever else the
+    call packs, at some speed on small calls.  Process-wide; returns the previous setting."""
+    return bool(_binding.vt_attn_set_split_keys(1 if enable else 0))
 
 
 def check_device_status(stream=None, device=None):

@@ -40,6 +40,7 @@ EXPORTED = (
     "vt_rope2d",
     "vt_attn_fwd_rope2d",
     "vt_attn_fwd_swa",
+    "vt_attn_set_split_keys",
     "vt_attn_status_string",
     "vt_attn_version",
 )
@@ -91,6 +92,8 @@ def _load():
     lib.vt_attn_status_string.restype = ctypes.c_char_p
     lib.vt_attn_version.argtypes = []
     lib.vt_attn_version.restype = I32
+    lib.vt_attn_set_split_keys.argtypes = [I32]
+    lib.vt_attn_set_split_keys.restype = I32
     return lib
 
 
@@ -192,3 +195,7 @@ def status_string(status: int) -> str:
 
 def vt_attn_version() -> int:
     return lib.vt_attn_version()
+
+
+def vt_attn_set_split_keys(enable: int) -> int:
+    return lib.vt_attn_set_split_keys(1 if enable else 0)

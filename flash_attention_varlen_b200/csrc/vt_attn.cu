@@ -3,6 +3,7 @@
 // Host side only: argument validation, the per-(device, stream) scratch
 // buffer that holds the work list, TMA descriptors for the bf16 kernel, and
 // the two launches of a call (scheduling prepass, then the attention kernel).
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -278,6 +279,8 @@ namespace {
 
 int sm_count();  // of the current device; 0 if it cannot be read
 
+std::atomic<int32_t> g_split_keys{1};  // vt_attn_set_split_keys
+
 // The forward of a validated call with the library-owned, per-(device, stream) work list.
 vt_status fwd_impl(const vt::FwdCall& c) {
   int dev = 0;
@@ -299,7 +302,8 @@ vt_status fwd_impl(const vt::FwdCall& c) {
   const long long fewest =
       (static_cast<long long>(c.total_tokens) + vt::kBf16BlockRows - 1) / vt::kBf16BlockRows * c.H;
   const int nsm = sm_count();
-  if (c.dtype == VT_DTYPE_BF16 && nsm > 1 && 2 * fewest <= nsm &&
+  if (c.dtype == VT_DTYPE_BF16 && g_split_keys.load(std::memory_order_relaxed) != 0 && nsm > 1 &&
+      2 * fewest <= nsm &&
       c.total_tokens > (vt::kSplitMinKeyTiles - 1) * 128) {
     if (sc->split_units < nsm / 2) {
       if (sc->split_ptr) {
@@ -635,5 +639,9 @@ const char* vt_attn_status_string(vt_status s) {
 }
 
 int32_t vt_attn_version(void) { return 100; }
+
+int32_t vt_attn_set_split_keys(int32_t enable) {
+  return g_split_keys.exchange(enable != 0 ? 1 : 0);
+}
 
 }  // extern "C"

@@ -304,6 +304,18 @@ vt_status vt_attn_fwd_swa(const void* q, const void* k, const void* v, void* out
                           int32_t Hq, int32_t Hkv, int32_t D, float scale, int32_t window,
                           void* stream);
 
+/*
+ * Whether bf16 calls of vt_attn_fwd and vt_attn_fwd_rope2d may split a unit's keys over
+ * two CTAs (enable != 0, the default) or never do (enable == 0).  A call with at most half
+ * as many (256-row block, head) units as SMs normally sums each row of a segment of at
+ * least four 128-key tiles in two halves, so its rows can differ in rounding from the
+ * same segment inside a larger call (both within the bf16 bound against the definition).
+ * With splitting off, a segment's output is the same bits whatever else the call packs,
+ * at the cost of speed on small calls.  Process-wide; takes effect for calls queued after
+ * it returns.  Returns the previous setting (1 or 0).
+ */
+int32_t vt_attn_set_split_keys(int32_t enable);
+
 /* Static, human-readable name of a status code. */
 const char* vt_attn_status_string(vt_status status);
 

@@ -174,3 +174,14 @@ def test_window_wrappers_validate_on_host(binding):
     perm = torch.arange(4, dtype=torch.int32)
     with pytest.raises(ValueError):
         fa.permute_rows(x, perm)                     # CPU tensors: the library is GPU-only
+
+
+def test_split_keys_option_round_trips(binding):
+    """vt_attn_set_split_keys is host state only: it returns the previous setting."""
+    prev = binding.vt_attn_set_split_keys(0)
+    try:
+        assert prev in (0, 1)
+        assert binding.vt_attn_set_split_keys(1) == 0
+        assert binding.vt_attn_set_split_keys(7) == 1  # any non-zero enables
+    finally:
+        binding.vt_attn_set_split_keys(prev)

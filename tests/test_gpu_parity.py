@@ -394,6 +394,22 @@ def test_split_key_units():
     assert not np.array_equal(alone, batch)  # the two really are different summation orders
 
 
+def test_split_keys_off_restores_batch_invariance_bitwise():
+    """With split-key units forbidden, a 700-token segment computed alone (a call small
+    enough to split) is the same bits as inside a 9000-token batch."""
+    import flash_attention_varlen_b200 as fa
+    big = workloads.Case("no_split", workloads.cu_from_lengths([700] + [1100] * 7 + [600]), seed=14,
+                         dtype="bf16")
+    bq, bk, bv = big.inputs()
+    batch = _run(bq, bk, bv, big.cu_seqlens, "bf16")[:700]
+    prev = fa.set_split_keys(False)
+    try:
+        alone = _run(bq[:700], bk[:700], bv[:700], np.array([0, 700], np.int32), "bf16")
+    finally:
+        fa.set_split_keys(prev)
+    assert np.array_equal(alone, batch)
+
+
 def test_deterministic():
     case = workloads.varlen8_case()
     q, k, v = case.inputs()
