@@ -73,3 +73,16 @@ def test_key_tile_periods_of_the_tower_layers():
     assert bench.key_tile_periods(window, 16, 148) == 7 * 8
     # fewer units than SMs: one unit per CTA
     assert bench.key_tile_periods(workloads.cu_from_lengths([1024]), 16, 148) == 8
+
+
+def test_measured_peaks_names_its_source(tmp_path, monkeypatch):
+    """The roofline's peak comes from MEASURED_PEAKS.json when present, else the stated
+    fallback, and the label says which."""
+    import json
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peak, hbm, src = bench.measured_peaks()
+    assert (peak, hbm) == (1590.0, 6650.0) and src.startswith("fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"bf16_tflops": 1608.2, "hbm_gbs": 6539.0}))
+    peak, hbm, src = bench.measured_peaks()
+    assert (peak, hbm) == (1608.2, 6539.0) and "MEASURED_PEAKS.json" in src and not src.startswith("fallback")
